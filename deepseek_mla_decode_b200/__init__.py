@@ -1,0 +1,184 @@
+"""B200-native weight-absorbed MLA decode.
+
+Thin Python binding over the C ABI of ``libmla.so`` (``include/mla_decode.h``): it only
+marshals torch tensors into pointers, sizes and the current CUDA stream.  Every step of
+the computation runs in the library's CUDA kernels; there is no fallback path, and a
+missing or unbuildable library raises ``RuntimeError``.
+
+    meta = get_metadata(cache_seqlens, s_q, H)
+    out, lse = decode(q_nope, q_pe, kv_cache, block_table, cache_seqlens,
+                      softmax_scale, causal, meta)
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmla.so")
+
+MLA_DEVICE_ERR_BLOCK_ID = 1
+MLA_DEVICE_ERR_SEQLEN = 2
+MLA_DEVICE_ERR_TIMEOUT = 4
+MLA_DEVICE_ERR_METADATA = 8
+
+EXPORTED_SYMBOLS = (
+    "mla_status_string",
+    "mla_metadata_size",
+    "mla_get_metadata",
+    "mla_workspace_size",
+    "mla_decode",
+    "mla_decode_attention",
+    "mla_decode_combine",
+    "mla_device_sm_count",
+)
+
+_lib = None
+
+
+class MLAError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn} failed: {status_string(code)} ({code})")
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmla.so (building it first if sources are newer) and declare signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path) or path == LIB_PATH:
+        try:
+            from . import build as _build
+
+            _build.build()
+        except Exception as e:  # pragma: no cover - build errors are reported loudly
+            if not os.path.exists(path):
+                raise RuntimeError(f"libmla.so is missing and could not be built: {e}") from e
+    L = ctypes.CDLL(path)
+    c_int, c_size, c_vp, c_i64, c_f = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
+    L.mla_status_string.restype = ctypes.c_char_p
+    L.mla_status_string.argtypes = [c_int]
+    L.mla_metadata_size.restype = c_int
+    L.mla_metadata_size.argtypes = [c_int, c_int, c_int, ctypes.POINTER(c_size)]
+    L.mla_workspace_size.restype = c_int
+    L.mla_workspace_size.argtypes = [c_int, c_int, c_int, ctypes.POINTER(c_size)]
+    L.mla_device_sm_count.restype = c_int
+    L.mla_device_sm_count.argtypes = [ctypes.POINTER(c_int)]
+    L.mla_get_metadata.restype = c_int
+    L.mla_get_metadata.argtypes = [c_vp, c_int, c_int, c_int, c_vp, c_size, c_vp]
+    dec_args = [c_vp, c_vp, c_vp, c_i64, c_vp, c_int, c_vp, c_int, c_int, c_int, c_f, c_int,
+                c_vp, c_size, c_vp, c_size, c_vp, c_vp, c_vp, c_vp]
+    for fn in (L.mla_decode, L.mla_decode_attention):
+        fn.restype = c_int
+        fn.argtypes = dec_args
+    L.mla_decode_combine.restype = c_int
+    L.mla_decode_combine.argtypes = [c_vp, c_int, c_int, c_int, c_int, c_vp, c_size, c_vp, c_size, c_vp, c_vp,
+                                     c_vp, c_vp]
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return load_library().mla_status_string(code).decode()
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise MLAError(fn, code)
+
+
+def metadata_size(B: int, s_q: int, H: int) -> int:
+    n = ctypes.c_size_t()
+    _check("mla_metadata_size", load_library().mla_metadata_size(B, s_q, H, ctypes.byref(n)))
+    return n.value
+
+
+def workspace_size(B: int, s_q: int, H: int) -> int:
+    n = ctypes.c_size_t()
+    _check("mla_workspace_size", load_library().mla_workspace_size(B, s_q, H, ctypes.byref(n)))
+    return n.value
+
+
+def device_sm_count() -> int:
+    n = ctypes.c_int()
+    _check("mla_device_sm_count", load_library().mla_device_sm_count(ctypes.byref(n)))
+    return n.value
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def get_metadata(cache_seqlens, s_q: int, H: int, metadata=None, stream=None):
+    """Split-KV schedule for one decode step (device int32 buffer)."""
+    import torch
+
+    B = cache_seqlens.shape[0]
+    nbytes = metadata_size(B, s_q, H)
+    if metadata is None:
+        metadata = torch.empty((nbytes + 3) // 4, dtype=torch.int32, device=cache_seqlens.device)
+    _check("mla_get_metadata", load_library().mla_get_metadata(
+        cache_seqlens.data_ptr(), B, s_q, H, metadata.data_ptr(), metadata.numel() * metadata.element_size(),
+        _stream_ptr(stream)))
+    return metadata
+
+
+def _decode_args(q_nope, q_pe, kv_cache, block_table, cache_seqlens, softmax_scale, causal, metadata, workspace,
+                 out, lse, status, stream):
+    B, s_q, H, _ = q_nope.shape
+    for name, t in (("q_nope", q_nope), ("q_pe", q_pe), ("kv_cache", kv_cache), ("block_table", block_table),
+                    ("cache_seqlens", cache_seqlens), ("out", out), ("lse", lse)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    return (q_nope.data_ptr(), q_pe.data_ptr(), kv_cache.data_ptr(), kv_cache.shape[0], block_table.data_ptr(),
+            block_table.shape[1], cache_seqlens.data_ptr(), B, s_q, H, float(softmax_scale), int(bool(causal)),
+            metadata.data_ptr(), metadata.numel() * metadata.element_size(), workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), out.data_ptr(), lse.data_ptr(),
+            status.data_ptr() if status is not None else None, _stream_ptr(stream))
+
+
+def _alloc_outputs(q_nope, workspace, out, lse):
+    import torch
+
+    B, s_q, H, _ = q_nope.shape
+    if workspace is None:
+        workspace = torch.empty(workspace_size(B, s_q, H), dtype=torch.uint8, device=q_nope.device)
+    if out is None:
+        out = torch.empty((B, s_q, H, 512), dtype=torch.bfloat16, device=q_nope.device)
+    if lse is None:
+        lse = torch.empty((B, s_q, H), dtype=torch.float32, device=q_nope.device)
+    return workspace, out, lse
+
+
+def decode(q_nope, q_pe, kv_cache, block_table, cache_seqlens, softmax_scale: float, causal: bool, metadata,
+           workspace=None, out=None, lse=None, status=None, stream=None) -> Tuple[object, object]:
+    """Weight-absorbed MLA decode; returns (out bf16 [B, s_q, H, 512], lse fp32 [B, s_q, H])."""
+    workspace, out, lse = _alloc_outputs(q_nope, workspace, out, lse)
+    _check("mla_decode", load_library().mla_decode(
+        *_decode_args(q_nope, q_pe, kv_cache, block_table, cache_seqlens, softmax_scale, causal, metadata,
+                      workspace, out, lse, status, stream)))
+    return out, lse
+
+
+def decode_attention(q_nope, q_pe, kv_cache, block_table, cache_seqlens, softmax_scale: float, causal: bool,
+                     metadata, workspace, out, lse, status=None, stream=None):
+    """The split-KV attention launch alone (see mla_decode_attention)."""
+    _check("mla_decode_attention", load_library().mla_decode_attention(
+        *_decode_args(q_nope, q_pe, kv_cache, block_table, cache_seqlens, softmax_scale, causal, metadata,
+                      workspace, out, lse, status, stream)))
+
+
+def decode_combine(cache_seqlens, max_blocks: int, s_q: int, H: int, metadata, workspace, out, lse, status=None,
+                   stream=None):
+    """The LSE-combine launch alone (see mla_decode_combine)."""
+    B = cache_seqlens.shape[0]
+    _check("mla_decode_combine", load_library().mla_decode_combine(
+        cache_seqlens.data_ptr(), int(max_blocks), B, s_q, H, metadata.data_ptr(),
+        metadata.numel() * metadata.element_size(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+        out.data_ptr(), lse.data_ptr(), status.data_ptr() if status is not None else None, _stream_ptr(stream)))

@@ -1,0 +1,305 @@
+// Host side of the C ABI declared in include/mla_decode.h: argument validation,
+// TMA tensor-map encoding and the launch sequence (schedule kernel; attention kernel +
+// LSE-combine kernel).  No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include "mla_internal.h"
+#include "../../include/mla_decode.h"
+
+namespace mla {
+cudaError_t launch_metadata(const int32_t* seqlens, int B, int s_q, int H, int num_workers, int32_t* meta,
+                            cudaStream_t stream);
+cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, int max_blocks, int B, int M,
+                           const float* part_o, const float* part_lse, void* out, float* lse,
+                           int32_t* status, cudaStream_t stream);
+cudaError_t decode_kernel_setup(int device);
+cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
+                          const int32_t* block_table, int max_blocks, const int32_t* seqlens,
+                          const int32_t* meta, int64_t num_blocks, int B, int s_q, int H, float scale,
+                          int causal, void* out, float* lse, float* part_o, float* part_lse,
+                          int32_t* status, int num_ctas, cudaStream_t stream);
+}  // namespace mla
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  bool ok = false;
+  int sm_count = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+
+// Per-device one-time setup: SM count, architecture check, kernel attributes.
+mla_status_t device_info(int* sm_count) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_DEVICE;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    d.ready = true;
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    if (major != 10 || minor != 0) return MLA_ERR_DEVICE;
+    if (mla::decode_kernel_setup(dev) != cudaSuccess) return MLA_ERR_CUDA;
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return MLA_ERR_CUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    d.sm_count = sms;
+    d.ok = true;
+  }
+  if (!d.ok) return MLA_ERR_DEVICE;
+  *sm_count = d.sm_count;
+  return MLA_OK;
+}
+
+bool shape_supported(int B, int s_q, int H) {
+  if (B < 1 || B > 65536) return false;
+  if (s_q < 1 || s_q > 4) return false;
+  return H == 16 || H == 32 || H == 64 || H == 128;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_workers_for(int sm_count) {
+  int w = sm_count / 2;
+  if (w > mla::kMaxWorkers) w = mla::kMaxWorkers;
+  return w < 1 ? 1 : w;
+}
+
+int parts_for(int num_workers, int s_q, int H) {
+  const int T = (s_q * H + mla::kRowsPerTile - 1) / mla::kRowsPerTile;
+  const int P = num_workers / T;
+  return P < 1 ? 1 : P;
+}
+
+bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+            const cuuint32_t* box) {
+  cuuint32_t es[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(mla_status_t s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_WORKSPACE_TOO_SMALL: return "MLA_ERR_WORKSPACE_TOO_SMALL";
+    case MLA_ERR_DEVICE: return "MLA_ERR_DEVICE";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+mla_status_t mla_metadata_size(int B, int s_q, int H, size_t* bytes) {
+  if (!bytes) return MLA_ERR_INVALID_ARG;
+  if (!shape_supported(B, s_q, H)) return MLA_ERR_UNSUPPORTED;
+  *bytes = static_cast<size_t>(mla::meta_words(B)) * sizeof(int32_t);
+  return MLA_OK;
+}
+
+mla_status_t mla_device_sm_count(int* sm_count) {
+  if (!sm_count) return MLA_ERR_INVALID_ARG;
+  return device_info(sm_count);
+}
+
+mla_status_t mla_workspace_size(int B, int s_q, int H, size_t* bytes) {
+  if (!bytes) return MLA_ERR_INVALID_ARG;
+  if (!shape_supported(B, s_q, H)) return MLA_ERR_UNSUPPORTED;
+  int sms = 0;
+  mla_status_t st = device_info(&sms);
+  if (st != MLA_OK) return st;
+  const int64_t slots = mla::ws_slots(B, num_workers_for(sms));
+  const int64_t M = static_cast<int64_t>(s_q) * H;
+  *bytes = static_cast<size_t>(slots * M * (mla::kDLatent + 1) * sizeof(float));
+  return MLA_OK;
+}
+
+mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int B, int s_q, int H, void* metadata,
+                              size_t metadata_bytes, void* stream) {
+  if (!cache_seqlens || !metadata) return MLA_ERR_INVALID_ARG;
+  if (!shape_supported(B, s_q, H)) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(metadata) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u)) return MLA_ERR_INVALID_ARG;
+  size_t need = 0;
+  mla_metadata_size(B, s_q, H, &need);
+  if (metadata_bytes < need) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  mla_status_t st = device_info(&sms);
+  if (st != MLA_OK) return st;
+  if (mla::launch_metadata(cache_seqlens, B, s_q, H, num_workers_for(sms), static_cast<int32_t*>(metadata),
+                           static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Shared validation of the decode arguments; fills the derived launch sizes.
+struct DecodeGeom {
+  int sms, workers, T, P, M;
+  int64_t slots;
+};
+
+mla_status_t check_decode_args(const void* q_nope, const void* q_pe, const void* kv_cache, int64_t num_blocks,
+                               const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens, int B,
+                               int s_q, int H, float softmax_scale, const void* metadata, size_t metadata_bytes,
+                               const void* workspace, size_t workspace_bytes, const void* out, const float* lse,
+                               const int32_t* status, DecodeGeom* g) {
+  if (!q_nope || !q_pe || !kv_cache || !block_table || !cache_seqlens || !metadata || !out || !lse)
+    return MLA_ERR_INVALID_ARG;
+  if (!shape_supported(B, s_q, H)) return MLA_ERR_UNSUPPORTED;
+  if (num_blocks < 1 || num_blocks > (int64_t)INT32_MAX || max_blocks < 1) return MLA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || softmax_scale > 1e30f) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_nope) || !aligned16(q_pe) || !aligned16(kv_cache) || !aligned16(out) || !aligned16(metadata) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(status) & 3u))
+    return MLA_ERR_INVALID_ARG;
+  size_t need_meta = 0, need_ws = 0;
+  mla_metadata_size(B, s_q, H, &need_meta);
+  if (metadata_bytes < need_meta) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  mla_status_t st = mla_workspace_size(B, s_q, H, &need_ws);
+  if (st != MLA_OK) return st;
+  if (workspace_bytes < need_ws) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (!workspace || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
+  st = device_info(&g->sms);
+  if (st != MLA_OK) return st;
+  g->M = s_q * H;
+  g->workers = num_workers_for(g->sms);
+  g->T = (g->M + mla::kRowsPerTile - 1) / mla::kRowsPerTile;
+  g->P = parts_for(g->workers, s_q, H);
+  g->slots = mla::ws_slots(B, g->workers);
+  return MLA_OK;
+}
+
+mla_status_t launch_attention(const void* q_nope, const void* q_pe, const void* kv_cache, int64_t num_blocks,
+                              const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens, int B,
+                              int s_q, int H, float softmax_scale, int causal, const void* metadata,
+                              void* workspace, void* out, float* lse, int32_t* status, const DecodeGeom& g,
+                              cudaStream_t s) {
+  const int64_t rows = static_cast<int64_t>(B) * g.M;
+  CUtensorMap tm_kv, tm_qn, tm_qp;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)mla::kDQK, (cuuint64_t)mla::kBlockSize, (cuuint64_t)num_blocks};
+    cuuint64_t strides[2] = {(cuuint64_t)mla::kDQK * 2, (cuuint64_t)mla::kDQK * 2 * mla::kBlockSize};
+    cuuint32_t box[3] = {64, 64, 1};
+    if (!encode(&tm_kv, kv_cache, 3, dims, strides, box)) return MLA_ERR_INVALID_ARG;
+  }
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)mla::kDLatent, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)mla::kDLatent * 2};
+    cuuint32_t box[2] = {64, 64};
+    if (!encode(&tm_qn, q_nope, 2, dims, strides, box)) return MLA_ERR_INVALID_ARG;
+  }
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)mla::kDRope, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)mla::kDRope * 2};
+    cuuint32_t box[2] = {64, 64};
+    if (!encode(&tm_qp, q_pe, 2, dims, strides, box)) return MLA_ERR_INVALID_ARG;
+  }
+  float* part_o = static_cast<float*>(workspace);
+  float* part_lse = part_o + g.slots * g.M * mla::kDLatent;
+  if (mla::launch_decode(tm_kv, tm_qn, tm_qp, block_table, max_blocks, cache_seqlens,
+                         static_cast<const int32_t*>(metadata), num_blocks, B, s_q, H, softmax_scale, causal != 0,
+                         out, lse, part_o, part_lse, status, 2 * g.P * g.T, s) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status_t mla_decode_attention(const void* q_nope, const void* q_pe, const void* kv_cache, int64_t num_blocks,
+                                  const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens, int B,
+                                  int s_q, int H, float softmax_scale, int causal, const void* metadata,
+                                  size_t metadata_bytes, void* workspace, size_t workspace_bytes, void* out,
+                                  float* lse, int32_t* status, void* stream) {
+  DecodeGeom g;
+  mla_status_t st = check_decode_args(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens,
+                                      B, s_q, H, softmax_scale, metadata, metadata_bytes, workspace,
+                                      workspace_bytes, out, lse, status, &g);
+  if (st != MLA_OK) return st;
+  return launch_attention(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, B, s_q, H,
+                          softmax_scale, causal, metadata, workspace, out, lse, status, g,
+                          static_cast<cudaStream_t>(stream));
+}
+
+mla_status_t mla_decode_combine(const int32_t* cache_seqlens, int max_blocks, int B, int s_q, int H,
+                                const void* metadata, size_t metadata_bytes, const void* workspace,
+                                size_t workspace_bytes, void* out, float* lse, int32_t* status, void* stream) {
+  if (!cache_seqlens || !metadata || !workspace || !out || !lse) return MLA_ERR_INVALID_ARG;
+  if (!shape_supported(B, s_q, H)) return MLA_ERR_UNSUPPORTED;
+  if (max_blocks < 1) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(metadata) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(status) & 3u))
+    return MLA_ERR_INVALID_ARG;
+  size_t need_meta = 0, need_ws = 0;
+  mla_metadata_size(B, s_q, H, &need_meta);
+  if (metadata_bytes < need_meta) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  mla_status_t st = mla_workspace_size(B, s_q, H, &need_ws);
+  if (st != MLA_OK) return st;
+  if (workspace_bytes < need_ws) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  st = device_info(&sms);
+  if (st != MLA_OK) return st;
+  const int M = s_q * H;
+  const int64_t slots = mla::ws_slots(B, num_workers_for(sms));
+  const float* part_o = static_cast<const float*>(workspace);
+  const float* part_lse = part_o + slots * M * mla::kDLatent;
+  if (mla::launch_combine(static_cast<const int32_t*>(metadata), cache_seqlens, max_blocks, B, M, part_o, part_lse,
+                          out, lse, status, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+mla_status_t mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, int64_t num_blocks,
+                        const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens, int B,
+                        int s_q, int H, float softmax_scale, int causal, const void* metadata,
+                        size_t metadata_bytes, void* workspace, size_t workspace_bytes, void* out, float* lse,
+                        int32_t* status, void* stream) {
+  DecodeGeom g;
+  mla_status_t st = check_decode_args(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens,
+                                      B, s_q, H, softmax_scale, metadata, metadata_bytes, workspace,
+                                      workspace_bytes, out, lse, status, &g);
+  if (st != MLA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_attention(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, B, s_q, H,
+                        softmax_scale, causal, metadata, workspace, out, lse, status, g, s);
+  if (st != MLA_OK) return st;
+  const float* part_o = static_cast<const float*>(workspace);
+  const float* part_lse = part_o + g.slots * g.M * mla::kDLatent;
+  if (mla::launch_combine(static_cast<const int32_t*>(metadata), cache_seqlens, max_blocks, B, g.M, part_o,
+                          part_lse, out, lse, status, s) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+}  // extern "C"

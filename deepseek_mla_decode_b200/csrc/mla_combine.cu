@@ -1,0 +1,107 @@
+// LSE-combine kernel: merges the normalised partial outputs of split sequences.
+//
+// A sequence cut into S pieces has, per query row, partial outputs O_s (each already
+// divided by its own softmax sum) and their log-sum-exps lse_s.  The exact merge is
+//     lse = ln sum_s exp(lse_s),      out = sum_s exp(lse_s - lse) * O_s
+// (split-K merge; "DeepSeek speed test / FA3" article, section 2.1 names the split and
+// the softmax_lse side output).  HBM-bound: one warp per query row streams the S
+// partial rows with 16-byte loads and writes the bf16 row once.
+//
+// The kernel also finishes rows the decode kernel does not own: sequences with no
+// visible key (out = 0, lse = -inf) and sequences with an invalid length (NaN and an
+// error bit in the status word).
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+#include "mla_internal.h"
+
+namespace mla {
+
+namespace {
+
+constexpr int kWarps = 8;
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(kWarps * 32) combine_kernel(
+    const int32_t* __restrict__ meta, const int32_t* __restrict__ seqlens, int max_blocks,
+    int B, int M, const float* __restrict__ part_o, const float* __restrict__ part_lse,
+    __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int32_t* status) {
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.y * kWarps + warp;
+  if (row >= M) return;
+  const int n = seqlens[b];
+  const int ns = meta[off_num_splits(B) + b];
+  uint2* orow = reinterpret_cast<uint2*>(out + ((int64_t)b * M + row) * kDLatent);
+  const bool bad_len = n < 0 || (int64_t)n > (int64_t)max_blocks * kBlockSize;
+  if (bad_len || ns == 0) {
+    const float v = bad_len ? __int_as_float(0x7fc00000) : 0.0f;
+    const uint32_t pv = pack_bf16x2(v, v);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) orow[k * 32 + lane] = make_uint2(pv, pv);
+    if (lane == 0) {
+      lse[(int64_t)b * M + row] = bad_len ? __int_as_float(0x7fc00000) : -INFINITY;
+      if (bad_len && row == 0 && status) atomicOr(status, kErrSeqlen);
+    }
+    return;
+  }
+  if (ns == 1) return;  // written by the decode kernel
+
+  const int64_t slot0 = meta[off_split_prefix(B) + b];
+  // pass 1: max and sum over the partial lse values (every lane redundantly)
+  float m = -INFINITY;
+  bool any_nan = false;
+  for (int s = 0; s < ns; ++s) {
+    const float l = part_lse[(slot0 + s) * M + row];
+    any_nan |= (l != l);
+    m = fmaxf(m, l);
+  }
+  float res_lse;
+  float4 acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (any_nan) {
+    res_lse = __int_as_float(0x7fc00000);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] = make_float4(res_lse, res_lse, res_lse, res_lse);
+  } else if (m == -INFINITY) {
+    res_lse = -INFINITY;
+  } else {
+    float z = 0.f;
+    for (int s = 0; s < ns; ++s) z += __expf(part_lse[(slot0 + s) * M + row] - m);
+    res_lse = m + __logf(z);
+    for (int s = 0; s < ns; ++s) {
+      const float w = __expf(part_lse[(slot0 + s) * M + row] - res_lse);
+      const float4* src = reinterpret_cast<const float4*>(part_o + ((slot0 + s) * M + row) * kDLatent);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 v = src[k * 32 + lane];
+        acc[k].x += w * v.x;
+        acc[k].y += w * v.y;
+        acc[k].z += w * v.z;
+        acc[k].w += w * v.w;
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    orow[k * 32 + lane] = make_uint2(pack_bf16x2(acc[k].x, acc[k].y), pack_bf16x2(acc[k].z, acc[k].w));
+  if (lane == 0) lse[(int64_t)b * M + row] = res_lse;
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, int max_blocks, int B,
+                           int M, const float* part_o, const float* part_lse, void* out, float* lse,
+                           int32_t* status, cudaStream_t stream) {
+  dim3 grid(B, (M + kWarps - 1) / kWarps);
+  combine_kernel<<<grid, kWarps * 32, 0, stream>>>(meta, seqlens, max_blocks, B, M, part_o, part_lse,
+                                                   reinterpret_cast<__nv_bfloat16*>(out), lse, status);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

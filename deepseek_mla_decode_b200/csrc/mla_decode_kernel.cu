@@ -1,0 +1,762 @@
+// Split-KV weight-absorbed MLA decode kernel for sm_100a.
+//
+// Math (weight-absorbed MLA: KsanaLLM 0.6.0 release notes, section 2.1; softmax scale
+// 1/sqrt(192): Paddle 3.0 inference article, long-sequence section; s_q > 1 draft
+// tokens with a causal mask among them: same article, speculative decoding):
+//     S = Q K^T,  Q = [q_nope | q_pe] (rows x 576),  K = cache rows (keys x 576)
+//     O = softmax(scale * S) V,  V = first 512 columns of the same cache rows
+//
+// Work unit: a 2-CTA cluster owns 128 query rows (row = token * H + head) of one
+// sequence piece (a contiguous block range from the split-KV schedule).  CTA r holds
+// rows [64r, 64r + 64) and accumulates their full 512-wide output in its TMEM.
+// Both GEMMs are cta_group::2 tcgen05 MMAs with M = 128 (64 rows per CTA), N = 256:
+//   QK: per 256-key tile, CTA r stages keys [128r, 128r + 128) of the tile (its half
+//       of the B operand) in 64-dim chunks; each CTA receives S for its 64 rows over
+//       all 256 keys (TMEM "2x2" layout: lanes 0-63 keys 0..127, lanes 64-127 keys
+//       128..255, 128 columns).
+//   PV: for each 256-wide half h of the output, CTA r stages V[key block, dims
+//       256h + 128r + (0..127)] (its half of N); each CTA receives O for its rows over
+//       all 256 dims of that half.
+// O uses TMEM columns [0, 256), the two S buffers [256, 384) and [384, 512).
+//
+// Warp roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer (leader CTA
+// only) and TMEM owner, warps 4..11 = softmax / correction / epilogue (thread = one
+// row x 64 keys of S, one row x 128 dims of O).  Every mbarrier wait is bounded; a
+// timeout sets MLA_DEVICE_ERR_TIMEOUT, raises a CTA-wide abort flag and the kernel
+// drains and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+#include "mla_internal.h"
+#include "ptx_sm100.cuh"
+
+namespace mla {
+
+using namespace ptx;
+
+namespace {
+
+constexpr int kNumThreads = 384;
+constexpr int kProducerWarp = 0;
+constexpr int kMmaWarp = 1;
+constexpr int kSoftmaxWarp0 = 4;
+constexpr int kNumSoftmaxThreads = 256;
+constexpr int kStages = 7;
+constexpr int kStageBytes = 16384;
+constexpr int kChunkBytes = 8192;  // one 64-row x 64-column bf16 SW128 box
+constexpr int kQChunks = 9;        // 576 / 64
+constexpr int kQBytes = kQChunks * kChunkBytes;
+constexpr int kPBytes = 4 * kChunkBytes;  // 64 rows x 256 keys bf16
+constexpr int kSmemQ = 0;
+constexpr int kSmemP = kSmemQ + kQBytes;
+constexpr int kSmemRing = kSmemP + kPBytes;
+constexpr int kSmemDyn = kSmemRing + kStages * kStageBytes;
+constexpr uint32_t kTmemO = 0, kTmemS0 = 256, kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only when the max grows by > 2^8
+constexpr uint32_t kIdescQK = make_idesc_bf16(128, 256, false, false);
+constexpr uint32_t kIdescPV = make_idesc_bf16(128, 256, false, true);
+constexpr int kBarSoftmax = 1;  // named barrier id for the 256 softmax threads
+
+struct Params {
+  CUtensorMap tm_kv;  // [num_blocks][64][576] bf16, box {64, 64, 1}, SW128
+  CUtensorMap tm_qn;  // [B*M][512] bf16, box {64, 64}, SW128
+  CUtensorMap tm_qp;  // [B*M][64] bf16, box {64, 64}, SW128
+  const int32_t* block_table;
+  const int32_t* seqlens;
+  const int32_t* meta;
+  __nv_bfloat16* out;
+  float* lse;
+  float* part_o;
+  float* part_lse;
+  int32_t* status;
+  int64_t num_blocks;
+  uint64_t timeout_ns;
+  int max_blocks;
+  int B, s_q, H, M;
+  float scale_log2;
+  int causal;
+};
+
+struct __align__(8) Ctrl {
+  uint64_t full[kStages];   // leader: stage landed in both CTAs (count 2 + tx)
+  uint64_t empty[kStages];  // both: stage consumed by the MMAs (commit)
+  uint64_t q_full;          // leader: Q of both CTAs landed (count 1 + tx)
+  uint64_t q_empty;         // both: last QK of the piece done (commit)
+  uint64_t s_full[2];       // both: S buffer written (commit)
+  uint64_t p_full;          // leader: P written in both CTAs (count 2)
+  uint64_t p_free;          // both: PV done (commit)
+  uint64_t o_free;          // leader: O read out by both CTAs (count 2)
+  uint64_t tail;            // both: local landing barrier of a stage that needs tail zeroing
+  uint32_t tmem_base;
+  volatile int abort;
+  float red_max[2][4][64];
+  float red_sum[4][64];   // sum of the bf16-rounded weights (normalises the output)
+  float red_sum32[4][64]; // sum of the fp32 weights (gives the lse)
+  int bad_piece;
+};
+
+struct Piece {
+  int b, k_lo, k_hi, split, n;
+};
+
+// Walks the pieces of one partition.  Pieces of sequences whose length is invalid
+// are skipped consistently by every role (the combine kernel writes their NaN rows).
+struct PieceWalker {
+  const Params* p;
+  int cb, ck, be, ke;
+  const int32_t* nblk;
+  const int32_t* first_part;
+  int part;
+  __device__ PieceWalker(const Params& prm, int part_) : p(&prm), part(part_) {
+    const int32_t* m = prm.meta;
+    cb = m[off_part_start() + 2 * part];
+    ck = m[off_part_start() + 2 * part + 1];
+    be = m[off_part_end() + 2 * part];
+    ke = m[off_part_end() + 2 * part + 1];
+    nblk = m + off_nblk();
+    first_part = m + off_first_part(prm.B);
+  }
+  __device__ bool next(Piece& pc) {
+    while (cb < p->B && (cb < be || (cb == be && ck < ke))) {
+      const int hi = (cb == be) ? ke : nblk[cb];
+      const int b = cb, lo = ck;
+      cb += 1;
+      ck = 0;
+      if (lo >= hi) continue;
+      const int n = p->seqlens[b];
+      if (n < 0 || (int64_t)n > (int64_t)p->max_blocks * kBlockSize) continue;
+      pc.b = b;
+      pc.k_lo = lo;
+      pc.k_hi = hi;
+      pc.split = part - first_part[b];
+      pc.n = n;
+      return true;
+    }
+    return false;
+  }
+};
+
+__device__ __forceinline__ int num_tiles(const Piece& pc) {
+  return (pc.k_hi - pc.k_lo + kBlocksPerTile - 1) / kBlocksPerTile;
+}
+__device__ __forceinline__ int blocks_in_tile(const Piece& pc, int t) {
+  const int r = pc.k_hi - pc.k_lo - t * kBlocksPerTile;
+  return r < kBlocksPerTile ? r : kBlocksPerTile;
+}
+// valid keys (< n) in block kb of tile t
+__device__ __forceinline__ int rows_in_block(const Piece& pc, int t, int kb) {
+  const int key0 = (pc.k_lo + t * kBlocksPerTile + kb) * kBlockSize;
+  const int r = pc.n - key0;
+  return r < kBlockSize ? r : kBlockSize;
+}
+
+__device__ __forceinline__ void set_status(const Params& p, int bits) {
+  if (p.status) atomicOr(p.status, bits);
+}
+
+// Bounded wait that also gives up when another role of this CTA aborted.
+__device__ __forceinline__ bool wait_bar(Ctrl* c, const Params& p, uint32_t bar, uint32_t parity,
+                                         bool cluster_scope) {
+  const bool ok0 = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+  if (ok0) return true;
+  const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i) {
+      const bool ok = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+      if (ok) return true;
+    }
+    if (c->abort) return false;
+    if (globaltimer_ns() > deadline) {
+      c->abort = 1;
+      set_status(p, kErrTimeout);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d_cg2(uint32_t dst, const void* tmap, uint32_t bar_cluster,
+                                                int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_cg2(uint32_t dst, const void* tmap, uint32_t bar_cluster,
+                                                int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void umma_2sm(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void commit_2sm(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)0x3)
+      : "memory");
+}
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+__device__ __forceinline__ int clamp_block_id(const Params& p, int32_t id) {
+  if (id < 0 || (int64_t)id >= p.num_blocks) {
+    set_status(p, kErrBlockId);
+    return 0;
+  }
+  return id;
+}
+
+// ===========================================================================
+// the kernel
+// ===========================================================================
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
+    mla_decode_kernel(const __grid_constant__ Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ Ctrl ctrl;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + kSmemQ, sP = sbase + kSmemP, sRing = sbase + kSmemRing;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int worker = blockIdx.x >> 1;
+  const int P = p.meta[kHdrNumParts];
+  int T = p.meta[kHdrNumTiles];
+  if (p.meta[kHdrMagic] != kMetaMagic || p.meta[kHdrB] != p.B || p.meta[kHdrSq] != p.s_q ||
+      p.meta[kHdrH] != p.H || P * T * 2 != (int)gridDim.x) {
+    if (tid == 0 && blockIdx.x == 0) set_status(p, kErrMetadata);
+    T = 0;  // every role skips; the CTA still joins the cluster barriers below
+  }
+  const int tile = worker / P;
+  const int part = worker % P;
+  const int tile_row0 = tile * kRowsPerTile;
+
+  // ---- setup ---------------------------------------------------------------
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&ctrl.full[s]), 2);
+      mbar_init(smem_u32(&ctrl.empty[s]), 1);
+    }
+    mbar_init(smem_u32(&ctrl.q_full), 1);
+    mbar_init(smem_u32(&ctrl.q_empty), 1);
+    mbar_init(smem_u32(&ctrl.s_full[0]), 1);
+    mbar_init(smem_u32(&ctrl.s_full[1]), 1);
+    mbar_init(smem_u32(&ctrl.p_full), 2);
+    mbar_init(smem_u32(&ctrl.p_free), 1);
+    mbar_init(smem_u32(&ctrl.o_free), 2);
+    mbar_init(smem_u32(&ctrl.tail), 1);
+    ctrl.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&ctrl.tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    prefetch_tmap(&p.tm_kv);
+    prefetch_tmap(&p.tm_qn);
+    prefetch_tmap(&p.tm_qp);
+  }
+  tc_fence_before();
+  __syncthreads();
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  tc_fence_after();
+  const uint32_t tmem = ctrl.tmem_base;
+
+  if (tile < T) {
+    // =======================================================================
+    // producer
+    // =======================================================================
+    if (warp == kProducerWarp) {
+      PieceWalker walk(p, part);
+      Piece pc;
+      uint32_t it = 0, tail_uses = 0;
+      int npieces = 0;
+      bool ok = true;
+      const uint32_t q_full_l = mapa_shared(smem_u32(&ctrl.q_full), 0);
+      // acquire a ring slot; returns slot index
+      auto acquire = [&](uint32_t& slot) -> bool {
+        slot = it % kStages;
+        const uint32_t use = it / kStages;
+        if (use > 0 && !wait_bar(&ctrl, p, smem_u32(&ctrl.empty[slot]), (use - 1) & 1, false)) return false;
+        return true;
+      };
+      while (ok && walk.next(pc)) {
+        const int64_t row_base = (int64_t)pc.b * p.M + tile_row0 + kRowsPerCta * (int)rank;
+        // ---- Q of this piece ----
+        if (lane == 0) {
+          if (npieces > 0) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.q_empty), (npieces - 1) & 1, false);
+          if (ok) {
+            if (leader) mbar_arrive_expect_tx(smem_u32(&ctrl.q_full), 2 * kQBytes);
+            for (int c = 0; c < kQChunks; ++c) {
+              if (c < 8)
+                tma_load_2d_cg2(sQ + c * kChunkBytes, &p.tm_qn, q_full_l, 64 * c, (int)row_base);
+              else
+                tma_load_2d_cg2(sQ + c * kChunkBytes, &p.tm_qp, q_full_l, 0, (int)row_base);
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        ++npieces;
+        const int nt = num_tiles(pc);
+        const int32_t* bt = p.block_table + (int64_t)pc.b * p.max_blocks;
+        // stage issue helpers (lane 0 issues; the whole warp joins tail zeroing)
+        auto issue_qk = [&](int t) {
+          const int nb = blocks_in_tile(pc, t);
+          const int own0 = 2 * (int)rank;
+          int ids[2];
+          int own = 0;
+          for (int i = 0; i < 2; ++i)
+            if (own0 + i < nb) ids[own++] = clamp_block_id(p, bt[pc.k_lo + t * kBlocksPerTile + own0 + i]);
+          for (int c = 0; c < kQChunks && ok; ++c) {
+            uint32_t slot;
+            if (lane == 0) ok = acquire(slot);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (lane == 0) {
+              const uint32_t fb = smem_u32(&ctrl.full[slot]);
+              if (leader)
+                mbar_arrive_expect_tx(fb, kChunkBytes * nb);
+              else
+                mbar_arrive_remote(mapa_shared(fb, 0));
+              const uint32_t fbl = mapa_shared(fb, 0);
+              for (int i = 0; i < own; ++i)
+                tma_load_3d_cg2(sRing + slot * kStageBytes + i * kChunkBytes, &p.tm_kv, fbl, 64 * c, 0, ids[i]);
+            }
+            ++it;
+          }
+        };
+        auto issue_pv = [&](int t) {
+          const int nb = blocks_in_tile(pc, t);
+          for (int h = 0; h < 2 && ok; ++h) {
+            for (int kb = 0; kb < nb && ok; ++kb) {
+              const int id = clamp_block_id(p, bt[pc.k_lo + t * kBlocksPerTile + kb]);
+              const int rv = rows_in_block(pc, t, kb);
+              const bool needs_tail = (rv & 15) != 0;  // a partial 16-key MMA step reads rows >= n
+              uint32_t slot;
+              if (lane == 0) ok = acquire(slot);
+              ok = __shfl_sync(0xffffffffu, ok, 0);
+              if (!ok) break;
+              slot = __shfl_sync(0xffffffffu, slot, 0);
+              const uint32_t dst = sRing + slot * kStageBytes;
+              const int d0 = 256 * h + 128 * (int)rank;
+              const uint32_t fb = smem_u32(&ctrl.full[slot]);
+              if (!needs_tail) {
+                if (lane == 0) {
+                  if (leader)
+                    mbar_arrive_expect_tx(fb, 2 * kStageBytes);
+                  else
+                    mbar_arrive_remote(mapa_shared(fb, 0));
+                  const uint32_t fbl = mapa_shared(fb, 0);
+                  tma_load_3d_cg2(dst, &p.tm_kv, fbl, d0, 0, id);
+                  tma_load_3d_cg2(dst + kChunkBytes, &p.tm_kv, fbl, d0 + 64, 0, id);
+                }
+              } else {
+                // Land locally, zero rows [rv, 64) of both boxes (NaN-safe: those rows
+                // meet P = 0 inside the last MMA step), then release to the leader.
+                const uint32_t tb = smem_u32(&ctrl.tail);
+                if (lane == 0) {
+                  mbar_arrive_expect_tx(tb, kStageBytes);
+                  tma_load_3d(dst, &p.tm_kv, tb, d0, 0, id);
+                  tma_load_3d(dst + kChunkBytes, &p.tm_kv, tb, d0 + 64, 0, id);
+                  ok = wait_bar(&ctrl, p, tb, tail_uses & 1, false);
+                }
+                ++tail_uses;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (ok) {
+                  // 2 boxes x (64 - rv) rows x 128 B, 16 B per store
+                  const int nvec = 2 * (kBlockSize - rv) * 8;
+                  for (int v = lane; v < nvec; v += 32) {
+                    const int box = v / ((kBlockSize - rv) * 8);
+                    const int rem = v % ((kBlockSize - rv) * 8);
+                    const uint32_t a = dst + box * kChunkBytes + (rv + rem / 8) * 128 + (rem % 8) * 16;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
+                  }
+                  fence_proxy_async_smem();
+                  __syncwarp();
+                  if (lane == 0) {
+                    if (leader)
+                      mbar_arrive(fb);
+                    else
+                      mbar_arrive_remote(mapa_shared(fb, 0));
+                  }
+                }
+              }
+              ++it;
+            }
+          }
+        };
+        for (int t = 0; t < nt && ok; ++t) {
+          issue_qk(t);
+          if (t >= 1) issue_pv(t - 1);
+        }
+        if (ok) issue_pv(nt - 1);
+      }
+    }
+    // =======================================================================
+    // MMA issuer (leader CTA only)
+    // =======================================================================
+    else if (warp == kMmaWarp && leader) {
+      PieceWalker walk(p, part);
+      Piece pc;
+      uint32_t it = 0, qk_count = 0, pv_count = 0;
+      int npieces = 0;
+      bool ok = true;
+      const bool elected = elect_one();
+      while (ok && walk.next(pc)) {
+        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.q_full), npieces & 1, true);
+        tc_fence_after();
+        const int nt = num_tiles(pc);
+        auto mma_qk = [&](int t) {
+          const uint32_t buf = qk_count & 1;
+          const uint32_t d = tmem + kTmemS0 + 128 * buf;
+          for (int c = 0; c < kQChunks && ok; ++c) {
+            const uint32_t slot = it % kStages;
+            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), (it / kStages) & 1, true);
+            if (!ok) break;
+            tc_fence_after();
+            if (elected) {
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t a = make_smem_desc(sQ + c * kChunkBytes + ks * 32, 16, 1024, kSwizzle128B);
+                const uint64_t b = make_smem_desc(sRing + slot * kStageBytes + ks * 32, 16, 1024, kSwizzle128B);
+                umma_2sm(d, a, b, kIdescQK, (c | ks) != 0);
+              }
+              commit_2sm(smem_u32(&ctrl.empty[slot]));
+            }
+            __syncwarp();
+            ++it;
+          }
+          if (elected && ok) {
+            commit_2sm(smem_u32(&ctrl.s_full[buf]));
+            if (t == nt - 1) commit_2sm(smem_u32(&ctrl.q_empty));
+          }
+          __syncwarp();
+          ++qk_count;
+        };
+        auto mma_pv = [&](int t) {
+          if (!ok) return;
+          ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_full), pv_count & 1, true);
+          if (ok && t == 0 && npieces > 0) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.o_free), (npieces - 1) & 1, true);
+          if (!ok) return;
+          tc_fence_after();
+          const int nb = blocks_in_tile(pc, t);
+          for (int h = 0; h < 2 && ok; ++h) {
+            for (int kb = 0; kb < nb && ok; ++kb) {
+              const uint32_t slot = it % kStages;
+              ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), (it / kStages) & 1, true);
+              if (!ok) break;
+              tc_fence_after();
+              const int rv = rows_in_block(pc, t, kb);
+              const int ksteps = (rv + 15) >> 4;
+              if (elected) {
+                for (int ks = 0; ks < ksteps; ++ks) {
+                  const uint64_t a = make_smem_desc(sP + kb * kChunkBytes + ks * 32, 16, 1024, kSwizzle128B);
+                  const uint64_t b = make_smem_desc(sRing + slot * kStageBytes + ks * 2048, 8192, 1024, kSwizzle128B);
+                  umma_2sm(tmem + kTmemO + 128 * h, a, b, kIdescPV, !(t == 0 && kb == 0 && ks == 0));
+                }
+                commit_2sm(smem_u32(&ctrl.empty[slot]));
+              }
+              __syncwarp();
+              ++it;
+            }
+          }
+          if (elected && ok) commit_2sm(smem_u32(&ctrl.p_free));
+          __syncwarp();
+          ++pv_count;
+        };
+        for (int t = 0; t < nt && ok; ++t) {
+          mma_qk(t);
+          if (t >= 1) mma_pv(t - 1);
+        }
+        mma_pv(nt - 1);
+        ++npieces;
+      }
+    }
+    // =======================================================================
+    // softmax / correction / epilogue
+    // =======================================================================
+    else if (warp >= kSoftmaxWarp0) {
+      const int st = tid - kSoftmaxWarp0 * 32;  // 0..255
+      const int g = st >> 7;                   // column group: keys 64g.. of each half; O half g
+      const int L = st & 127;                  // TMEM lane
+      const int quad = (warp & 3);             // lane quadrant this warp may access
+      const int m = L & 63;                    // row within the CTA
+      const int hk = L >> 6;                   // key half (0: keys 0..127, 1: 128..255)
+      const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+      const int grow = tile_row0 + kRowsPerCta * (int)rank + m;  // row within the sequence
+      const bool row_valid = grow < p.M;
+      const int token = row_valid ? grow / p.H : 0;
+      const uint32_t p_full_l = mapa_shared(smem_u32(&ctrl.p_full), 0);
+      const uint32_t o_free_l = mapa_shared(smem_u32(&ctrl.o_free), 0);
+      PieceWalker walk(p, part);
+      Piece pc;
+      uint32_t qk_count = 0, pv_count = 0;
+      bool ok = true;
+      while (ok && walk.next(pc)) {
+        const int nt = num_tiles(pc);
+        const int piece_end = min(pc.n, pc.k_hi * kBlockSize);
+        int lim = p.causal ? (pc.n - p.s_q + token) : (pc.n - 1);
+        lim = min(lim, piece_end - 1);
+        if (!row_valid) lim = -1;
+        // l_part: sum of the bf16 weights that enter the PV MMA (output normaliser, so
+        // the weights sum to one exactly); l32_part: fp32 weights (the lse).
+        float m_used = -INFINITY, l_part = 0.f, l32_part = 0.f;
+        for (int t = 0; t < nt && ok; ++t) {
+          const uint32_t buf = qk_count & 1;
+          ok = wait_bar(&ctrl, p, smem_u32(&ctrl.s_full[buf]), (qk_count >> 1) & 1, false);
+          if (!ok) break;
+          tc_fence_after();
+          uint32_t sr[64];
+          {
+            uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+            uint32_t (&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+            const uint32_t ta = tmem + kTmemS0 + 128 * buf + lane_off + 64 * g;
+            tmem_ld32(ta, a);
+            tmem_ld32(ta + 32, b);
+            tmem_wait_ld();
+          }
+          const int key0 = (pc.k_lo + t * kBlocksPerTile) * kBlockSize + 128 * hk + 64 * g;
+          int cnt = lim - key0 + 1;
+          cnt = cnt < 0 ? 0 : (cnt > 64 ? 64 : cnt);
+          float lmax = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const float x = __uint_as_float(sr[c]) * p.scale_log2;
+            sr[c] = __float_as_uint(x);
+            if (c < cnt) lmax = fmaxf(lmax, x);
+          }
+          ctrl.red_max[qk_count & 1][2 * hk + g][m] = lmax;
+          named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
+          float rmax = ctrl.red_max[qk_count & 1][0][m];
+          rmax = fmaxf(rmax, ctrl.red_max[qk_count & 1][1][m]);
+          rmax = fmaxf(rmax, ctrl.red_max[qk_count & 1][2][m]);
+          rmax = fmaxf(rmax, ctrl.red_max[qk_count & 1][3][m]);
+          const float m_new = fmaxf(m_used, rmax);
+          const bool rescale = m_new > m_used + kRescaleThreshold;
+          float alpha = 1.f;
+          if (rescale) {
+            alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_new);
+            m_used = m_new;
+            l_part *= alpha;
+            l32_part *= alpha;
+          }
+          const float mref = (m_used == -INFINITY) ? 0.f : m_used;
+          uint32_t pk[32];
+          float lsum = 0.f, lsum32 = 0.f;
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const float e0 = (c < cnt) ? fast_exp2(__uint_as_float(sr[c]) - mref) : 0.f;
+            const float e1 = (c + 1 < cnt) ? fast_exp2(__uint_as_float(sr[c + 1]) - mref) : 0.f;
+            const uint32_t v = pack_bf16x2(e0, e1);
+            pk[c >> 1] = v;
+            lsum += bf16lo(v) + bf16hi(v);
+            lsum32 += e0 + e1;
+          }
+          l_part += lsum;
+          l32_part += lsum32;
+          // PV of the previous tile must be done before P is overwritten / O rescaled.
+          if (t >= 1) {
+            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1, false);
+            if (!ok) break;
+            ++pv_count;
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, rescale)) {
+              const uint32_t to = tmem + kTmemO + 128 * g + lane_off;
+#pragma unroll 1
+              for (int c = 0; c < 128; c += 32) {
+                uint32_t o[32];
+                tmem_ld32(to + c, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                asm volatile(
+                    "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+                    "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+                    "%29, %30, %31, %32};" ::"r"(to + c),
+                    "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7]),
+                    "r"(o[8]), "r"(o[9]), "r"(o[10]), "r"(o[11]), "r"(o[12]), "r"(o[13]), "r"(o[14]),
+                    "r"(o[15]), "r"(o[16]), "r"(o[17]), "r"(o[18]), "r"(o[19]), "r"(o[20]), "r"(o[21]),
+                    "r"(o[22]), "r"(o[23]), "r"(o[24]), "r"(o[25]), "r"(o[26]), "r"(o[27]), "r"(o[28]),
+                    "r"(o[29]), "r"(o[30]), "r"(o[31])
+                    : "memory");
+              }
+              tmem_wait_st();
+            }
+          }
+          // P -> shared memory: chunk (2 hk + g) holds keys 64 (2hk+g) .. of all 64 rows,
+          // K-major 128-byte swizzle (16-byte granule j of row m at j ^ (m & 7)).
+          {
+            const uint32_t prow = sP + (2 * hk + g) * kChunkBytes + m * 128;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint32_t a = prow + ((j ^ (m & 7)) << 4);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * j]), "r"(pk[4 * j + 1]),
+                           "r"(pk[4 * j + 2]), "r"(pk[4 * j + 3])
+                           : "memory");
+            }
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
+          if (st == 0) {
+            if (leader)
+              mbar_arrive(smem_u32(&ctrl.p_full));
+            else
+              mbar_arrive_remote(p_full_l);
+          }
+          ++qk_count;
+        }
+        if (!ok) break;
+        // ---- epilogue of the piece ----------------------------------------
+        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1, false);
+        if (!ok) break;
+        ++pv_count;
+        tc_fence_after();
+        ctrl.red_sum[2 * hk + g][m] = l_part;
+        ctrl.red_sum32[2 * hk + g][m] = l32_part;
+        if (st == 0) ctrl.bad_piece = 0;
+        named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
+        {
+          const int32_t* bt = p.block_table + (int64_t)pc.b * p.max_blocks;
+          int bad = 0;
+          for (int k = pc.k_lo + st; k < pc.k_hi; k += kNumSoftmaxThreads) {
+            const int32_t id = bt[k];
+            bad |= (id < 0 || (int64_t)id >= p.num_blocks);
+          }
+          if (bad) ctrl.bad_piece = 1;
+        }
+        const float l_row = ctrl.red_sum[0][m] + ctrl.red_sum[1][m] + ctrl.red_sum[2][m] + ctrl.red_sum[3][m];
+        const float l32_row =
+            ctrl.red_sum32[0][m] + ctrl.red_sum32[1][m] + ctrl.red_sum32[2][m] + ctrl.red_sum32[3][m];
+        named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
+        const bool bad = ctrl.bad_piece != 0;
+        const int nsplit = p.meta[off_num_splits(p.B) + pc.b];
+        const bool direct = (nsplit == 1);
+        const float nanf_ = __int_as_float(0x7fc00000);
+        const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
+        const float lse_val =
+            bad ? nanf_ : ((l32_row > 0.f) ? (m_used + __log2f(l32_row)) * 0.69314718055994531f : -INFINITY);
+        const int dim0 = 256 * g + 128 * hk;
+        const int64_t orow = (int64_t)pc.b * p.M + grow;
+        const int64_t slot = (int64_t)p.meta[off_split_prefix(p.B) + pc.b] + pc.split;
+        const uint32_t to = tmem + kTmemO + 128 * g + lane_off;
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(to + c, o);
+          tmem_wait_ld();
+          if (row_valid) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = bad ? nanf_ : __uint_as_float(o[j]) * inv_l;
+            if (direct) {
+              uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDLatent + dim0 + c);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                                    pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+            } else {
+              float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * p.M + grow) * kDLatent + dim0 + c);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            }
+          }
+        }
+        if (row_valid && hk == 0 && g == 0) {
+          if (direct)
+            p.lse[orow] = lse_val;
+          else
+            p.part_lse[slot * p.M + grow] = lse_val;
+        }
+        tc_fence_before();
+        named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
+        if (st == 0) {
+          if (leader)
+            mbar_arrive(smem_u32(&ctrl.o_free));
+          else
+            mbar_arrive_remote(o_free_l);
+        }
+      }
+    }
+  }
+
+  // ---- teardown ------------------------------------------------------------
+  tc_fence_before();
+  __syncthreads();
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  tc_fence_after();
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+}  // namespace
+
+struct DecodeLaunch {
+  CUtensorMap tm_kv, tm_qn, tm_qp;
+};
+
+cudaError_t decode_kernel_setup(int device) {
+  (void)device;
+  return cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDyn + 1024);
+}
+
+cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
+                          const int32_t* block_table, int max_blocks, const int32_t* seqlens,
+                          const int32_t* meta, int64_t num_blocks, int B, int s_q, int H, float scale,
+                          int causal, void* out, float* lse, float* part_o, float* part_lse,
+                          int32_t* status, int num_ctas, cudaStream_t stream) {
+  Params prm;
+  prm.tm_kv = tm_kv;
+  prm.tm_qn = tm_qn;
+  prm.tm_qp = tm_qp;
+  prm.block_table = block_table;
+  prm.seqlens = seqlens;
+  prm.meta = meta;
+  prm.out = reinterpret_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.part_o = part_o;
+  prm.part_lse = part_lse;
+  prm.status = status;
+  prm.num_blocks = num_blocks;
+  prm.timeout_ns = 1000000000ull;
+  prm.max_blocks = max_blocks;
+  prm.B = B;
+  prm.s_q = s_q;
+  prm.H = H;
+  prm.M = s_q * H;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.causal = causal;
+  mla_decode_kernel<<<num_ctas, kNumThreads, kSmemDyn + 1024, stream>>>(prm);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

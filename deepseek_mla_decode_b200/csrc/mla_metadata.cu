@@ -1,0 +1,180 @@
+// Split-KV scheduler: one CTA turns cache_seqlens into the partition schedule that
+// the decode kernel and the combine kernel follow.  Integer-only; the float64 oracle
+// states the same algorithm and the tests compare the two word for word.
+//
+// Cost model: every 64-row block costs 1 and every sequence with at least one block
+// costs kSchedOverheadBlocks more, placed before its first block.  pre[b] is the cost
+// of the sequences before b, so block k of sequence b sits at position
+// pre[b] + overhead + k.  With P partitions per row tile and
+// cap = max(kSchedMinCap, ceil(total / P)), block (b, k) belongs to partition
+// floor(position / cap): contiguous, near-equal ranges.  (Split-K parallelism is named
+// in the "DeepSeek speed test / FA3" article, section 2.1; this cost model is ours.)
+#include <cuda_runtime.h>
+#include <cstdint>
+#include "mla_internal.h"
+
+namespace mla {
+
+namespace {
+
+constexpr int kThreads = 1024;
+
+// Block-wide exclusive scan of int64 values held one per thread; returns the
+// exclusive prefix for this thread and writes the block total to *total.
+__device__ int64_t block_exclusive_scan(int64_t v, int64_t* scratch /*[32]*/, int64_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int64_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int64_t w = (lane < (kThreads / 32)) ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    scratch[lane] = w;  // inclusive warp totals
+  }
+  __syncthreads();
+  const int64_t warp_excl = (warp == 0) ? 0 : scratch[warp - 1];
+  *total = scratch[kThreads / 32 - 1];
+  __syncthreads();
+  return warp_excl + x - v;
+}
+
+__global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __restrict__ seqlens, int B,
+                                                            int s_q, int H, int num_workers,
+                                                            int32_t* __restrict__ meta) {
+  __shared__ int64_t scratch[32];
+  __shared__ int64_t s_carry, s_total;
+  const int tid = threadIdx.x;
+  const int M = s_q * H;
+  const int T = (M + kRowsPerTile - 1) / kRowsPerTile;
+  int P = num_workers / T;
+  if (P < 1) P = 1;
+
+  int32_t* part_start = meta + off_part_start();
+  int32_t* part_end = meta + off_part_end();
+  int32_t* nblk_out = meta + off_nblk();
+  int32_t* first_part = meta + off_first_part(B);
+  int32_t* num_splits = meta + off_num_splits(B);
+  int32_t* split_prefix = meta + off_split_prefix(B);
+
+  // ---- pass 1: total cost -------------------------------------------------
+  int64_t total = 0;
+  for (int base = 0; base < B; base += kThreads) {
+    const int b = base + tid;
+    int64_t cost = 0;
+    if (b < B) {
+      const int n = seqlens[b];
+      const int nb = n > 0 ? (n + kBlockSize - 1) / kBlockSize : 0;
+      nblk_out[b] = nb;
+      cost = nb > 0 ? nb + kSchedOverheadBlocks : 0;
+    }
+    int64_t t;
+    block_exclusive_scan(cost, scratch, &t);
+    total += t;
+  }
+  int64_t cap = (total + P - 1) / P;
+  if (cap < kSchedMinCap) cap = kSchedMinCap;
+
+  // default partition starts: past the end
+  for (int p = tid; p < kMaxWorkers; p += kThreads) {
+    part_start[2 * p] = B;
+    part_start[2 * p + 1] = 0;
+  }
+  if (tid == 0) s_carry = 0;
+  __syncthreads();
+
+  // ---- pass 2: per-sequence splits and partition starts -------------------
+  for (int base = 0; base < B; base += kThreads) {
+    const int b = base + tid;
+    int64_t cost = 0;
+    int nb = 0;
+    if (b < B) {
+      const int n = seqlens[b];
+      nb = n > 0 ? (n + kBlockSize - 1) / kBlockSize : 0;
+      cost = nb > 0 ? nb + kSchedOverheadBlocks : 0;
+    }
+    int64_t chunk_total;
+    const int64_t pre = s_carry + block_exclusive_scan(cost, scratch, &chunk_total);
+    if (b < B) {
+      if (nb > 0) {
+        const int64_t first_pos = pre + kSchedOverheadBlocks;
+        const int64_t p0 = first_pos / cap;
+        const int64_t p1 = (first_pos + nb - 1) / cap;
+        first_part[b] = (int32_t)p0;
+        num_splits[b] = (int32_t)(p1 - p0 + 1);
+        // partitions whose start position falls in [pre, pre + cost)
+        const int64_t lo = (pre + cap - 1) / cap;
+        const int64_t hi = (pre + cost - 1) / cap;
+        for (int64_t p = lo; p <= hi && p < P; ++p) {
+          const int64_t k = p * cap - first_pos;
+          part_start[2 * p] = b;
+          part_start[2 * p + 1] = (int32_t)(k > 0 ? k : 0);
+        }
+      } else {
+        first_part[b] = 0;
+        num_splits[b] = 0;
+      }
+    }
+    __syncthreads();
+    if (tid == 0) s_carry += chunk_total;
+    __syncthreads();
+  }
+
+  // ---- pass 3: split prefix ------------------------------------------------
+  if (tid == 0) s_carry = 0;
+  __syncthreads();
+  for (int base = 0; base < B; base += kThreads) {
+    const int b = base + tid;
+    const int64_t v = (b < B) ? num_splits[b] : 0;
+    int64_t chunk_total;
+    const int64_t ex = s_carry + block_exclusive_scan(v, scratch, &chunk_total);
+    if (b < B) split_prefix[b] = (int32_t)ex;
+    __syncthreads();
+    if (tid == 0) s_carry += chunk_total;
+    __syncthreads();
+  }
+  if (tid == 0) s_total = s_carry;
+  __syncthreads();
+
+  // ---- partition ends + header ---------------------------------------------
+  for (int p = tid; p < kMaxWorkers; p += kThreads) {
+    if (p + 1 < P) {
+      part_end[2 * p] = part_start[2 * (p + 1)];
+      part_end[2 * p + 1] = part_start[2 * (p + 1) + 1];
+    } else {
+      part_end[2 * p] = B;
+      part_end[2 * p + 1] = 0;
+    }
+  }
+  if (tid == 0) {
+    meta[kHdrMagic] = kMetaMagic;
+    meta[kHdrB] = B;
+    meta[kHdrSq] = s_q;
+    meta[kHdrH] = H;
+    meta[kHdrNumParts] = P;
+    meta[kHdrNumTiles] = T;
+    meta[kHdrCap] = (int32_t)cap;
+    meta[kHdrTotalSlots] = (int32_t)s_total;
+    meta[kHdrNumWorkers] = num_workers;
+    meta[kHdrOverhead] = kSchedOverheadBlocks;
+    for (int i = kHdrOverhead + 1; i < kHdrWords; ++i) meta[i] = 0;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_metadata(const int32_t* seqlens, int B, int s_q, int H, int num_workers,
+                            int32_t* meta, cudaStream_t stream) {
+  metadata_kernel<<<1, kThreads, 0, stream>>>(seqlens, B, s_q, H, num_workers, meta);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -1,0 +1,163 @@
+/*
+ * mla_decode.h -- C ABI of libmla.so: weight-absorbed multi-head latent attention
+ * (MLA) decode over a paged latent KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  For sequence b with n_b = cache_seqlens[b] cached tokens, query
+ * token i (0 <= i < s_q) and head h, the cache row of token t is
+ *     r_t = kv_cache[block_table[b][t / 64]][t % 64][0:576]  =  [ c_kv (512) | k_pe (64) ]
+ * and the key t is visible when t < n_b and, with causal != 0, t <= n_b - s_q + i
+ * (the s_q new tokens are the last s_q cache positions).  Over the visible keys:
+ *     s_t            = softmax_scale * (q_nope[b,i,h,:] . c_kv_t + q_pe[b,i,h,:] . k_pe_t)
+ *     lse[b,i,h]     = ln sum_t exp(s_t)
+ *     out[b,i,h,:]   = sum_t exp(s_t - lse) * c_kv_t
+ * Rows with no visible key get out = 0 and lse = -inf.
+ *
+ * Sources (page titles and sections): weight-absorbed MLA in decode, one latent row
+ * shared by all heads -- KsanaLLM 0.6.0 release notes, section 2.1 (WA-MLA / DP
+ * attention); softmax scale 1/sqrt(192) from DeepSeek's 192-wide attention head --
+ * Paddle 3.0 inference upgrade article, long-sequence (SageAttention) section;
+ * several draft tokens per sequence in one decode call -- same article, speculative
+ * decoding section; softmax_lse side output and split-K (split-KV) parallelism --
+ * "DeepSeek speed test / FA3" article, section 2.1; paged cache with a block table --
+ * Dewu deployment slides (PagedAttention) and the same FA3 article, section 4.1.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, contiguous
+ *    row-major in the shapes shown, and 16-byte aligned.  The library allocates
+ *    no device memory and keeps no state except a per-device cache of the SM count
+ *    and of kernel attributes.
+ *  - Calls that take a stream are asynchronous on that stream.  Host-detectable
+ *    errors are returned before anything is launched; nothing else is written.
+ *  - Device-detectable data errors (a block id outside [0, num_blocks) among the
+ *    blocks a sequence uses, n_b < 0, n_b > max_blocks * 64) never fault: the
+ *    affected sequence's out rows and lse are set to NaN and a bit is OR-ed into
+ *    *status (MLA_DEVICE_ERR_*) when status != NULL.  A bounded wait inside a
+ *    kernel that runs out (1 s) sets MLA_DEVICE_ERR_TIMEOUT and the kernel returns.
+ *  - No C++ exception crosses this boundary.  Calls are re-entrant given distinct
+ *    metadata / workspace buffers.
+ */
+#ifndef MLA_DECODE_H_
+#define MLA_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,         /* null pointer, negative size, misalignment, ... */
+  MLA_ERR_UNSUPPORTED = 2,         /* shape outside the supported set (see below)    */
+  MLA_ERR_CUDA = 3,                /* a CUDA runtime / driver call failed            */
+  MLA_ERR_WORKSPACE_TOO_SMALL = 4, /* metadata or workspace buffer below its size    */
+  MLA_ERR_DEVICE = 5               /* no sm_100 device current                        */
+} mla_status_t;
+
+/* Bits OR-ed into the optional device status word by the kernels. */
+#define MLA_DEVICE_ERR_BLOCK_ID 1 /* block_table entry outside [0, num_blocks) */
+#define MLA_DEVICE_ERR_SEQLEN 2   /* cache_seqlens[b] < 0 or > max_blocks * 64  */
+#define MLA_DEVICE_ERR_TIMEOUT 4  /* an internal bounded wait ran out           */
+#define MLA_DEVICE_ERR_METADATA 8 /* metadata not produced for these B, s_q, H   */
+
+/* Fixed geometry. */
+#define MLA_BLOCK_SIZE 64  /* cache rows per physical block   */
+#define MLA_D_LATENT 512   /* c_kv width = output width       */
+#define MLA_D_ROPE 64      /* k_pe / q_pe width               */
+#define MLA_D_QK 576       /* cache row width                 */
+
+/* Supported shapes: H in {16, 32, 64, 128}, s_q in {1, 2, 3, 4}, 1 <= B <= 65536. */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* mla_status_string(mla_status_t status);
+
+/*
+ * Bytes of the schedule buffer mla_get_metadata writes for (B, s_q, H).  Host only,
+ * no device call.  *bytes receives the size.
+ */
+mla_status_t mla_metadata_size(int B, int s_q, int H, size_t* bytes);
+
+/*
+ * Split-KV schedule for one decode step (shared by every layer of that step).
+ *
+ * The concatenation of all sequences' 64-row blocks is cut into contiguous ranges of
+ * near-equal cost, one per partition; every sequence also costs a fixed overhead
+ * before its first block.  A sequence cut across partitions is computed as several
+ * partial results that mla_decode merges by log-sum-exp (split-K parallelism, "DeepSeek
+ * speed test / FA3" article section 2.1; the cost model is this library's own).
+ *
+ *   cache_seqlens  device int32 [B]   (n_b; negative values count as 0 here)
+ *   metadata       device buffer of at least mla_metadata_size(B, s_q, H) bytes,
+ *                  written asynchronously on `stream`; opaque to the caller.
+ * The schedule depends only on (cache_seqlens, s_q, H, the device's SM count).
+ */
+mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int B, int s_q, int H,
+                              void* metadata, size_t metadata_bytes, void* stream);
+
+/*
+ * Upper bound, in bytes, of the fp32 scratch mla_decode needs for split partial
+ * results (partial outputs and their lse) for (B, s_q, H) on the current device.
+ */
+mla_status_t mla_workspace_size(int B, int s_q, int H, size_t* bytes);
+
+/*
+ * The decode attention itself.
+ *
+ *   q_nope         bf16 [B, s_q, H, 512]   absorbed latent queries
+ *   q_pe           bf16 [B, s_q, H, 64]    RoPE queries
+ *   kv_cache       bf16 [num_blocks, 64, 576]
+ *   block_table    int32 [B, max_blocks]   physical block of logical block k of b;
+ *                                          entries past ceil(n_b / 64) are never read
+ *   cache_seqlens  int32 [B]               n_b, counting the s_q new tokens
+ *   softmax_scale  scale applied to the scores (1/sqrt(192) for DeepSeek MLA)
+ *   causal         nonzero: causal mask among the s_q new tokens (bottom-right)
+ *   metadata       from mla_get_metadata for the same cache_seqlens, s_q, H
+ *   workspace      >= mla_workspace_size(B, s_q, H) bytes of device scratch
+ *   out            bf16 [B, s_q, H, 512]   (written)
+ *   lse            fp32 [B, s_q, H]        natural-log log-sum-exp of the scaled scores
+ *   status         device int32 (may be NULL): MLA_DEVICE_ERR_* bits are OR-ed in
+ *   stream         cudaStream_t (NULL = legacy default stream)
+ *
+ * Launches the split-KV attention kernel (one 2-CTA cluster per 128 query rows and
+ * partition; TMA-fed tcgen05 MMAs with TMEM accumulators) and then the LSE-combine
+ * kernel that merges split sequences.
+ */
+mla_status_t mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache,
+                        int64_t num_blocks, const int32_t* block_table, int max_blocks,
+                        const int32_t* cache_seqlens, int B, int s_q, int H,
+                        float softmax_scale, int causal, const void* metadata,
+                        size_t metadata_bytes, void* workspace, size_t workspace_bytes,
+                        void* out, float* lse, int32_t* status, void* stream);
+
+/*
+ * The two launches mla_decode performs, exposed separately (same arguments, same
+ * semantics; mla_decode == mla_decode_attention followed by mla_decode_combine on
+ * the same stream with the same workspace).
+ *
+ * mla_decode_attention: the split-KV attention kernel.  Sequences processed in one
+ *   piece get their out / lse rows written directly; pieces of split sequences write
+ *   normalised fp32 partial outputs and their lse into the workspace.
+ * mla_decode_combine: the LSE-combine kernel (split-K merge, "DeepSeek speed test /
+ *   FA3" article section 2.1): for every split sequence, lse = ln sum_s exp(lse_s) and
+ *   out = sum_s exp(lse_s - lse) O_s; it also writes the rows of sequences with no
+ *   visible key (0 / -inf) and of sequences with an invalid length (NaN).
+ */
+mla_status_t mla_decode_attention(const void* q_nope, const void* q_pe, const void* kv_cache,
+                                  int64_t num_blocks, const int32_t* block_table, int max_blocks,
+                                  const int32_t* cache_seqlens, int B, int s_q, int H,
+                                  float softmax_scale, int causal, const void* metadata,
+                                  size_t metadata_bytes, void* workspace, size_t workspace_bytes,
+                                  void* out, float* lse, int32_t* status, void* stream);
+mla_status_t mla_decode_combine(const int32_t* cache_seqlens, int max_blocks, int B, int s_q, int H,
+                                const void* metadata, size_t metadata_bytes, const void* workspace,
+                                size_t workspace_bytes, void* out, float* lse, int32_t* status,
+                                void* stream);
+
+/* Number of streaming multiprocessors the schedule targets on the current device. */
+mla_status_t mla_device_sm_count(int* sm_count);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_DECODE_H_ */
