@@ -32,6 +32,7 @@ EXPORTED_SYMBOLS = (
     "mla_decode",
     "mla_decode_attention",
     "mla_decode_combine",
+    "mla_decode_noalloc",
     "mla_device_sm_count",
 )
 
@@ -74,6 +75,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for fn in (L.mla_decode, L.mla_decode_attention):
         fn.restype = c_int
         fn.argtypes = dec_args
+    L.mla_decode_noalloc.restype = c_int
+    L.mla_decode_noalloc.argtypes = [c_vp, c_vp, c_vp, c_i64, c_vp, c_int, c_vp, c_int, c_int, c_int, c_f, c_int,
+                                     c_vp, c_size, c_vp, c_vp, c_vp, c_vp]
     L.mla_decode_combine.restype = c_int
     L.mla_decode_combine.argtypes = [c_vp, c_int, c_int, c_int, c_int, c_vp, c_size, c_vp, c_size, c_vp, c_vp,
                                      c_vp, c_vp]
@@ -182,3 +186,16 @@ def decode_combine(cache_seqlens, max_blocks: int, s_q: int, H: int, metadata, w
         cache_seqlens.data_ptr(), int(max_blocks), B, s_q, H, metadata.data_ptr(),
         metadata.numel() * metadata.element_size(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
         out.data_ptr(), lse.data_ptr(), status.data_ptr() if status is not None else None, _stream_ptr(stream)))
+
+
+def decode_noalloc(q_nope, q_pe, kv_cache, block_table, cache_seqlens, softmax_scale: float, causal: bool,
+                   metadata, out, lse, status=None, stream=None):
+    """mla_decode_noalloc: the decode with the library's built-in 64 MiB scratch instead
+    of a workspace, for callers that cannot allocate device memory.  ``out`` and ``lse``
+    are caller-provided.  Raises MLAError(code 4) when the shape needs more scratch."""
+    args = _decode_args(q_nope, q_pe, kv_cache, block_table, cache_seqlens, softmax_scale, causal, metadata,
+                        metadata, out, lse, status, stream)
+    # drop the workspace pointer / size (positions 14, 15) from the mla_decode argument list
+    args = args[:14] + args[16:]
+    _check("mla_decode_noalloc", load_library().mla_decode_noalloc(*args))
+    return out, lse

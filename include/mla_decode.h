@@ -154,6 +154,34 @@ mla_status_t mla_decode_combine(const int32_t* cache_seqlens, int max_blocks, in
                                 size_t workspace_bytes, void* out, float* lse, int32_t* status,
                                 void* stream);
 
+/*
+ * mla_decode without a caller-provided workspace, for callers that cannot allocate
+ * device memory (an engine whose memory pool already reserved the device, a plugin
+ * that only receives input and output pointers, a decode loop that cannot afford
+ * cudaMalloc's implicit synchronisation).  There is no counterpart of this call in
+ * the source pages; it is a deployment convenience.
+ *
+ * Same arguments and results as mla_decode minus the workspace.  The split-KV
+ * scratch is a 64 MiB array compiled into the library (each GPU that loads the
+ * library holds it until the process exits).  The call allocates nothing.
+ *  - If mla_workspace_size(B, s_q, H) exceeds 64 MiB it returns
+ *    MLA_ERR_WORKSPACE_TOO_SMALL and launches nothing (use mla_decode with your own
+ *    workspace for such shapes; for H = 128, s_q = 1 the limit is B <= 181 on a
+ *    148-SM B200).
+ *  - The first call on each device looks up the array's device address (with that
+ *    device current) and caches it; make that first call before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents; every slot
+ *    a call reads is written earlier in the same call, so nothing needs clearing.
+ *    Calls whose kernels overlap on the GPU (different streams without ordering)
+ *    race on the array: serialise them.
+ */
+mla_status_t mla_decode_noalloc(const void* q_nope, const void* q_pe, const void* kv_cache,
+                                int64_t num_blocks, const int32_t* block_table, int max_blocks,
+                                const int32_t* cache_seqlens, int B, int s_q, int H,
+                                float softmax_scale, int causal, const void* metadata,
+                                size_t metadata_bytes, void* out, float* lse, int32_t* status,
+                                void* stream);
+
 /* Number of streaming multiprocessors the schedule targets on the current device. */
 mla_status_t mla_device_sm_count(int* sm_count);
 
