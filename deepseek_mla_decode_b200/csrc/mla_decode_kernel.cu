@@ -79,7 +79,7 @@ struct Params {
 };
 
 struct __align__(8) Ctrl {
-  uint64_t full[kStages];   // leader: stage landed in both CTAs (count 2 + tx)
+  uint64_t full[kStages];   // leader: stage landed in both CTAs (count 1 + tx of both CTAs)
   uint64_t empty[kStages];  // both: stage consumed by the MMAs (commit)
   uint64_t q_full;          // leader: Q of both CTAs landed (count 1 + tx)
   uint64_t q_empty;         // both: last QK of the piece done (commit)
@@ -88,13 +88,16 @@ struct __align__(8) Ctrl {
   uint64_t p_free;          // both: PV done (commit)
   uint64_t o_free;          // leader: O read out by both CTAs (count 2)
   uint64_t tail;            // both: local landing barrier of a stage that needs tail zeroing
+  uint64_t peer_tail[kStages];  // leader: the peer zeroed its copy of the tail stage in this slot
   uint32_t tmem_base;
   volatile int abort;
   float red_max[2][4][64];
   float red_sum[4][64];   // sum of the bf16-rounded weights (normalises the output)
   float red_sum32[4][64]; // sum of the fp32 weights (gives the lse)
   int bad_piece;
+  int block_ids[128];  // producer's window of the current piece's physical block ids
 };
+constexpr int kIdRing = 128;
 
 struct Piece {
   int b, k_lo, k_hi, split, n;
@@ -258,7 +261,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
   // ---- setup ---------------------------------------------------------------
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&ctrl.full[s]), 2);
+      mbar_init(smem_u32(&ctrl.full[s]), 1);
       mbar_init(smem_u32(&ctrl.empty[s]), 1);
     }
     mbar_init(smem_u32(&ctrl.q_full), 1);
@@ -269,6 +272,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     mbar_init(smem_u32(&ctrl.p_free), 1);
     mbar_init(smem_u32(&ctrl.o_free), 2);
     mbar_init(smem_u32(&ctrl.tail), 1);
+    for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&ctrl.peer_tail[s]), 1);
     ctrl.abort = 0;
     fence_mbar_init();
   }
@@ -327,25 +331,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         ++npieces;
         const int nt = num_tiles(pc);
         const int32_t* bt = p.block_table + (int64_t)pc.b * p.max_blocks;
+        // Physical block ids of the piece, fetched 32 at a time (one coalesced load per
+        // lane) one chunk ahead of use into a 128-entry window; invalid ids are clamped
+        // to block 0 here (the epilogue turns that piece's rows into NaN).
+        const int piece_blocks = pc.k_hi - pc.k_lo;
+        auto fetch_id = [&](int i) -> int {
+          return (i < piece_blocks) ? clamp_block_id(p, bt[pc.k_lo + i]) : 0;
+        };
+        int id_pending = fetch_id(lane);
+        int id_chunks = 0;  // chunks of 32 ids stored in the window
+        auto ensure_ids = [&](int last) {  // make relative blocks <= last readable
+          while (last >= 32 * id_chunks) {
+            ctrl.block_ids[(32 * id_chunks + lane) % kIdRing] = id_pending;
+            ++id_chunks;
+            id_pending = fetch_id(32 * id_chunks + lane);
+            __syncwarp();
+          }
+        };
         // stage issue helpers (lane 0 issues; the whole warp joins tail zeroing)
         auto issue_qk = [&](int t) {
           const int nb = blocks_in_tile(pc, t);
           const int own0 = 2 * (int)rank;
+          ensure_ids(t * kBlocksPerTile + nb - 1);
           int ids[2];
           int own = 0;
           for (int i = 0; i < 2; ++i)
-            if (own0 + i < nb) ids[own++] = clamp_block_id(p, bt[pc.k_lo + t * kBlocksPerTile + own0 + i]);
+            if (own0 + i < nb) ids[own++] = ctrl.block_ids[(t * kBlocksPerTile + own0 + i) % kIdRing];
+          // Every stage must carry bytes from both CTAs: the leader's full barrier then
+          // cannot complete before the peer has issued the stage, which keeps the peer
+          // producer within one ring cycle of the MMAs (otherwise its empty-barrier
+          // parity could alias).  A peer without keys in this tile loads a copy of the
+          // tile's first block; those S columns are masked.
+          if (own == 0) ids[own++] = ctrl.block_ids[(t * kBlocksPerTile) % kIdRing];
+          const int peer_boxes = nb > 2 ? nb - 2 : 1;
+          const int lead_boxes = nb < 2 ? nb : 2;
           for (int c = 0; c < kQChunks && ok; ++c) {
             uint32_t slot;
             if (lane == 0) ok = acquire(slot);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             if (lane == 0) {
+              // Only the leader arrives (posting both CTAs' bytes); the peer's TMA
+              // completes its bytes on the leader's barrier.
               const uint32_t fb = smem_u32(&ctrl.full[slot]);
-              if (leader)
-                mbar_arrive_expect_tx(fb, kChunkBytes * nb);
-              else
-                mbar_arrive_remote(mapa_shared(fb, 0));
+              if (leader) mbar_arrive_expect_tx(fb, kChunkBytes * (lead_boxes + peer_boxes));
               const uint32_t fbl = mapa_shared(fb, 0);
               for (int i = 0; i < own; ++i)
                 tma_load_3d_cg2(sRing + slot * kStageBytes + i * kChunkBytes, &p.tm_kv, fbl, 64 * c, 0, ids[i]);
@@ -357,7 +386,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           const int nb = blocks_in_tile(pc, t);
           for (int h = 0; h < 2 && ok; ++h) {
             for (int kb = 0; kb < nb && ok; ++kb) {
-              const int id = clamp_block_id(p, bt[pc.k_lo + t * kBlocksPerTile + kb]);
+              const int id = ctrl.block_ids[(t * kBlocksPerTile + kb) % kIdRing];
               const int rv = rows_in_block(pc, t, kb);
               const bool needs_tail = (rv & 15) != 0;  // a partial 16-key MMA step reads rows >= n
               uint32_t slot;
@@ -370,10 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
               const uint32_t fb = smem_u32(&ctrl.full[slot]);
               if (!needs_tail) {
                 if (lane == 0) {
-                  if (leader)
-                    mbar_arrive_expect_tx(fb, 2 * kStageBytes);
-                  else
-                    mbar_arrive_remote(mapa_shared(fb, 0));
+                  if (leader) mbar_arrive_expect_tx(fb, 2 * kStageBytes);
                   const uint32_t fbl = mapa_shared(fb, 0);
                   tma_load_3d_cg2(dst, &p.tm_kv, fbl, d0, 0, id);
                   tma_load_3d_cg2(dst + kChunkBytes, &p.tm_kv, fbl, d0 + 64, 0, id);
@@ -403,9 +429,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
                   __syncwarp();
                   if (lane == 0) {
                     if (leader)
-                      mbar_arrive(fb);
+                      mbar_arrive(fb);  // the stage's only arrival, no bytes
                     else
-                      mbar_arrive_remote(mapa_shared(fb, 0));
+                      mbar_arrive_remote(mapa_shared(smem_u32(&ctrl.peer_tail[slot]), 0));
                   }
                 }
               }
@@ -426,7 +452,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     else if (warp == kMmaWarp && leader) {
       PieceWalker walk(p, part);
       Piece pc;
-      uint32_t it = 0, qk_count = 0, pv_count = 0;
+      uint32_t it = 0, qk_count = 0, pv_count = 0, tail_par = 0;
       int npieces = 0;
       bool ok = true;
       const bool elected = elect_one();
@@ -472,9 +498,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
             for (int kb = 0; kb < nb && ok; ++kb) {
               const uint32_t slot = it % kStages;
               ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), (it / kStages) & 1, true);
+              const int rv = rows_in_block(pc, t, kb);
+              if (ok && (rv & 15) != 0) {  // tail stage: the peer zeroes its copy too
+                ok = wait_bar(&ctrl, p, smem_u32(&ctrl.peer_tail[slot]), (tail_par >> slot) & 1, true);
+                tail_par ^= 1u << slot;
+              }
               if (!ok) break;
               tc_fence_after();
-              const int rv = rows_in_block(pc, t, kb);
               const int ksteps = (rv + 15) >> 4;
               if (elected) {
                 for (int ks = 0; ks < ksteps; ++ks) {
@@ -529,6 +559,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         // l_part: sum of the bf16 weights that enter the PV MMA (output normaliser, so
         // the weights sum to one exactly); l32_part: fp32 weights (the lse).
         float m_used = -INFINITY, l_part = 0.f, l32_part = 0.f;
+        // Block-id validity of the piece (loads issued now, consumed at the epilogue).
+        int bad_ids = 0;
+        {
+          const int32_t* bt = p.block_table + (int64_t)pc.b * p.max_blocks;
+          for (int k = pc.k_lo + st; k < pc.k_hi; k += kNumSoftmaxThreads) {
+            const int32_t id = bt[k];
+            bad_ids |= (id < 0 || (int64_t)id >= p.num_blocks);
+          }
+        }
         for (int t = 0; t < nt && ok; ++t) {
           const uint32_t buf = qk_count & 1;
           ok = wait_bar(&ctrl, p, smem_u32(&ctrl.s_full[buf]), (qk_count >> 1) & 1, false);
@@ -644,15 +683,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         ctrl.red_sum32[2 * hk + g][m] = l32_part;
         if (st == 0) ctrl.bad_piece = 0;
         named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
-        {
-          const int32_t* bt = p.block_table + (int64_t)pc.b * p.max_blocks;
-          int bad = 0;
-          for (int k = pc.k_lo + st; k < pc.k_hi; k += kNumSoftmaxThreads) {
-            const int32_t id = bt[k];
-            bad |= (id < 0 || (int64_t)id >= p.num_blocks);
-          }
-          if (bad) ctrl.bad_piece = 1;
-        }
+        if (bad_ids) ctrl.bad_piece = 1;
         const float l_row = ctrl.red_sum[0][m] + ctrl.red_sum[1][m] + ctrl.red_sum[2][m] + ctrl.red_sum[3][m];
         const float l32_row =
             ctrl.red_sum32[0][m] + ctrl.red_sum32[1][m] + ctrl.red_sum32[2][m] + ctrl.red_sum32[3][m];
