@@ -19,9 +19,10 @@
 //       all 256 dims of that half.
 // O uses TMEM columns [0, 256), the two S buffers [256, 384) and [384, 512).
 //
-// Warp roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer (leader CTA
-// only) and TMEM owner, warps 4..11 = softmax / correction / epilogue (thread = one
-// row x 64 keys of S, one row x 128 dims of O).  Every mbarrier wait is bounded; a
+// Warp roles (384 threads): warps 0, 2, 3 = TMA producers (alternate ring stages),
+// warp 1 = MMA issuer (leader CTA only) and TMEM owner, warps 4..11 = softmax /
+// correction / epilogue (thread = one row x 64 keys of S, one row x 128 dims of O).
+// Every mbarrier wait is bounded; a
 // timeout sets MLA_DEVICE_ERR_TIMEOUT, raises a CTA-wide abort flag and the kernel
 // drains and returns.
 #include <cuda.h>
@@ -38,7 +39,7 @@ using namespace ptx;
 namespace {
 
 constexpr int kNumThreads = 384;
-constexpr int kProducerWarp = 0;
+constexpr int kNumProducers = 3;  // warps 0, 2, 3
 constexpr int kMmaWarp = 1;
 constexpr int kSoftmaxWarp0 = 4;
 constexpr int kNumSoftmaxThreads = 256;
@@ -87,7 +88,7 @@ struct __align__(8) Ctrl {
   uint64_t p_full;          // leader: P written in both CTAs (count 2)
   uint64_t p_free;          // both: PV done (commit)
   uint64_t o_free;          // leader: O read out by both CTAs (count 2)
-  uint64_t tail;            // both: local landing barrier of a stage that needs tail zeroing
+  uint64_t tail[3];         // both: per-producer landing barrier of a stage that needs tail zeroing
   uint64_t peer_tail[kStages];  // leader: the peer zeroed its copy of the tail stage in this slot
   uint32_t tmem_base;
   volatile int abort;
@@ -95,7 +96,7 @@ struct __align__(8) Ctrl {
   float red_sum[4][64];   // sum of the bf16-rounded weights (normalises the output)
   float red_sum32[4][64]; // sum of the fp32 weights (gives the lse)
   int bad_piece;
-  int block_ids[128];  // producer's window of the current piece's physical block ids
+  int block_ids[3][128];  // each producer's window of the current piece's physical block ids
 };
 constexpr int kIdRing = 128;
 
@@ -271,7 +272,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     mbar_init(smem_u32(&ctrl.p_full), 2);
     mbar_init(smem_u32(&ctrl.p_free), 1);
     mbar_init(smem_u32(&ctrl.o_free), 2);
-    mbar_init(smem_u32(&ctrl.tail), 1);
+    for (int i = 0; i < 3; ++i) mbar_init(smem_u32(&ctrl.tail[i]), 1);
     for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&ctrl.peer_tail[s]), 1);
     ctrl.abort = 0;
     fence_mbar_init();
@@ -283,7 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
-  if (warp == kProducerWarp && lane == 0) {
+  if (warp == 0 && lane == 0) {
     prefetch_tmap(&p.tm_kv);
     prefetch_tmap(&p.tm_qn);
     prefetch_tmap(&p.tm_qp);
@@ -296,16 +297,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
 
   if (tile < T) {
     // =======================================================================
-    // producer
+    // producers: warps 0, 2 and 3 own ring stages k % 3 == 0, 1, 2 (one issuing
+    // warp sustains only ~half the L2 -> SM bandwidth a CTA needs; several warps
+    // issuing alternate stages of the same ring lift that limit).  Warp 0 also loads Q.
     // =======================================================================
-    if (warp == kProducerWarp) {
+    if (warp == 0 || warp == 2 || warp == 3) {
+      const int pi = (warp == 0) ? 0 : warp - 1;
+      int32_t* idwin = ctrl.block_ids[pi];
+      const uint32_t tb = smem_u32(&ctrl.tail[pi]);
       PieceWalker walk(p, part);
       Piece pc;
       uint32_t it = 0, tail_uses = 0;
       int npieces = 0;
       bool ok = true;
       const uint32_t q_full_l = mapa_shared(smem_u32(&ctrl.q_full), 0);
-      // acquire a ring slot; returns slot index
+      auto mine = [&]() { return (int)(it % kNumProducers) == pi; };
+      // acquire the ring slot of stage `it` (lane 0)
       auto acquire = [&](uint32_t& slot) -> bool {
         slot = it % kStages;
         const uint32_t use = it / kStages;
@@ -315,7 +322,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
       while (ok && walk.next(pc)) {
         const int64_t row_base = (int64_t)pc.b * p.M + tile_row0 + kRowsPerCta * (int)rank;
         // ---- Q of this piece ----
-        if (lane == 0) {
+        if (pi == 0 && lane == 0) {
           if (npieces > 0) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.q_empty), (npieces - 1) & 1, false);
           if (ok) {
             if (leader) mbar_arrive_expect_tx(smem_u32(&ctrl.q_full), 2 * kQBytes);
@@ -332,8 +339,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         const int nt = num_tiles(pc);
         const int32_t* bt = p.block_table + (int64_t)pc.b * p.max_blocks;
         // Physical block ids of the piece, fetched 32 at a time (one coalesced load per
-        // lane) one chunk ahead of use into a 128-entry window; invalid ids are clamped
-        // to block 0 here (the epilogue turns that piece's rows into NaN).
+        // lane) one chunk ahead of use into this warp's 128-entry window; invalid ids
+        // are clamped to block 0 here (the epilogue turns that piece's rows into NaN).
         const int piece_blocks = pc.k_hi - pc.k_lo;
         auto fetch_id = [&](int i) -> int {
           return (i < piece_blocks) ? clamp_block_id(p, bt[pc.k_lo + i]) : 0;
@@ -342,13 +349,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         int id_chunks = 0;  // chunks of 32 ids stored in the window
         auto ensure_ids = [&](int last) {  // make relative blocks <= last readable
           while (last >= 32 * id_chunks) {
-            ctrl.block_ids[(32 * id_chunks + lane) % kIdRing] = id_pending;
+            idwin[(32 * id_chunks + lane) % kIdRing] = id_pending;
             ++id_chunks;
             id_pending = fetch_id(32 * id_chunks + lane);
             __syncwarp();
           }
         };
-        // stage issue helpers (lane 0 issues; the whole warp joins tail zeroing)
         auto issue_qk = [&](int t) {
           const int nb = blocks_in_tile(pc, t);
           const int own0 = 2 * (int)rank;
@@ -356,29 +362,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           int ids[2];
           int own = 0;
           for (int i = 0; i < 2; ++i)
-            if (own0 + i < nb) ids[own++] = ctrl.block_ids[(t * kBlocksPerTile + own0 + i) % kIdRing];
+            if (own0 + i < nb) ids[own++] = idwin[(t * kBlocksPerTile + own0 + i) % kIdRing];
           // Every stage must carry bytes from both CTAs: the leader's full barrier then
           // cannot complete before the peer has issued the stage, which keeps the peer
-          // producer within one ring cycle of the MMAs (otherwise its empty-barrier
+          // producers within one ring cycle of the MMAs (otherwise its empty-barrier
           // parity could alias).  A peer without keys in this tile loads a copy of the
           // tile's first block; those S columns are masked.
-          if (own == 0) ids[own++] = ctrl.block_ids[(t * kBlocksPerTile) % kIdRing];
+          if (own == 0) ids[own++] = idwin[(t * kBlocksPerTile) % kIdRing];
           const int peer_boxes = nb > 2 ? nb - 2 : 1;
           const int lead_boxes = nb < 2 ? nb : 2;
           for (int c = 0; c < kQChunks && ok; ++c) {
+            if (!mine()) {
+              ++it;
+              continue;
+            }
             uint32_t slot;
             if (lane == 0) ok = acquire(slot);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            if (lane == 0) {
-              // Only the leader arrives (posting both CTAs' bytes); the peer's TMA
-              // completes its bytes on the leader's barrier.
-              const uint32_t fb = smem_u32(&ctrl.full[slot]);
-              if (leader) mbar_arrive_expect_tx(fb, kChunkBytes * (lead_boxes + peer_boxes));
-              const uint32_t fbl = mapa_shared(fb, 0);
-              for (int i = 0; i < own; ++i)
-                tma_load_3d_cg2(sRing + slot * kStageBytes + i * kChunkBytes, &p.tm_kv, fbl, 64 * c, 0, ids[i]);
-            }
+            slot = __shfl_sync(0xffffffffu, slot, 0);
+            // Only the leader arrives (posting both CTAs' bytes); the peer's TMA
+            // completes its bytes on the leader's barrier.
+            const uint32_t fb = smem_u32(&ctrl.full[slot]);
+            if (lane == 0 && leader) mbar_arrive_expect_tx(fb, kChunkBytes * (lead_boxes + peer_boxes));
+            if (lane < own)
+              tma_load_3d_cg2(sRing + slot * kStageBytes + lane * kChunkBytes, &p.tm_kv, mapa_shared(fb, 0), 64 * c,
+                              0, ids[lane]);
             ++it;
           }
         };
@@ -386,7 +395,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           const int nb = blocks_in_tile(pc, t);
           for (int h = 0; h < 2 && ok; ++h) {
             for (int kb = 0; kb < nb && ok; ++kb) {
-              const int id = ctrl.block_ids[(t * kBlocksPerTile + kb) % kIdRing];
+              if (!mine()) {
+                ++it;
+                continue;
+              }
+              const int id = idwin[(t * kBlocksPerTile + kb) % kIdRing];
               const int rv = rows_in_block(pc, t, kb);
               const bool needs_tail = (rv & 15) != 0;  // a partial 16-key MMA step reads rows >= n
               uint32_t slot;
@@ -398,16 +411,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
               const int d0 = 256 * h + 128 * (int)rank;
               const uint32_t fb = smem_u32(&ctrl.full[slot]);
               if (!needs_tail) {
-                if (lane == 0) {
-                  if (leader) mbar_arrive_expect_tx(fb, 2 * kStageBytes);
-                  const uint32_t fbl = mapa_shared(fb, 0);
-                  tma_load_3d_cg2(dst, &p.tm_kv, fbl, d0, 0, id);
-                  tma_load_3d_cg2(dst + kChunkBytes, &p.tm_kv, fbl, d0 + 64, 0, id);
-                }
+                if (lane == 0 && leader) mbar_arrive_expect_tx(fb, 2 * kStageBytes);
+                if (lane < 2)
+                  tma_load_3d_cg2(dst + lane * kChunkBytes, &p.tm_kv, mapa_shared(fb, 0), d0 + 64 * lane, 0, id);
               } else {
                 // Land locally, zero rows [rv, 64) of both boxes (NaN-safe: those rows
                 // meet P = 0 inside the last MMA step), then release to the leader.
-                const uint32_t tb = smem_u32(&ctrl.tail);
                 if (lane == 0) {
                   mbar_arrive_expect_tx(tb, kStageBytes);
                   tma_load_3d(dst, &p.tm_kv, tb, d0, 0, id);
