@@ -17,7 +17,7 @@ import os
 from typing import Optional, Tuple
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmla.so")
+LIB_PATH = os.environ.get("MLA_LIBRARY") or os.path.join(_HERE, "libmla.so")
 
 MLA_DEVICE_ERR_BLOCK_ID = 1
 MLA_DEVICE_ERR_SEQLEN = 2
@@ -50,7 +50,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(path) or path == LIB_PATH:
+    if not os.path.exists(path) or path == os.path.join(_HERE, "libmla.so"):
         try:
             from . import build as _build
 

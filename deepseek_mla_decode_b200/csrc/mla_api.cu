@@ -16,7 +16,8 @@ cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, int max_
                            const float* part_o, const float* part_lse, void* out, float* lse,
                            int32_t* status, cudaStream_t stream);
 cudaError_t decode_kernel_setup(int device);
-cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
+cudaError_t launch_decode(const void* kv_base, const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
+                          const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
                           const int32_t* block_table, int max_blocks, const int32_t* seqlens,
                           const int32_t* meta, int64_t num_blocks, int B, int s_q, int H, float scale,
                           int causal, void* out, float* lse, float* part_o, float* part_lse,
@@ -95,7 +96,7 @@ int parts_for(int num_workers, int s_q, int H) {
 
 bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
             const cuuint32_t* box) {
-  cuuint32_t es[3] = {1, 1, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -205,12 +206,21 @@ mla_status_t launch_attention(const void* q_nope, const void* q_pe, const void* 
                               void* workspace, void* out, float* lse, int32_t* status, const DecodeGeom& g,
                               cudaStream_t s) {
   const int64_t rows = static_cast<int64_t>(B) * g.M;
-  CUtensorMap tm_kv, tm_qn, tm_qp;
+  CUtensorMap tm_kv, tm_kv2, tm_qn, tm_qp;
   {
     cuuint64_t dims[3] = {(cuuint64_t)mla::kDQK, (cuuint64_t)mla::kBlockSize, (cuuint64_t)num_blocks};
     cuuint64_t strides[2] = {(cuuint64_t)mla::kDQK * 2, (cuuint64_t)mla::kDQK * 2 * mla::kBlockSize};
     cuuint32_t box[3] = {64, 64, 1};
     if (!encode(&tm_kv, kv_cache, 3, dims, strides, box)) return MLA_ERR_INVALID_ARG;
+  }
+  {
+    // The same cache viewed as [block][chunk of 64 columns][row][64]: one box of
+    // {64, 64 rows, 2 chunks} lands a 64-row x 128-column slab as two stacked
+    // 128-byte-swizzled 64x64 tiles with a single TMA instruction.
+    cuuint64_t dims[4] = {64, (cuuint64_t)mla::kBlockSize, (cuuint64_t)(mla::kDQK / 64), (cuuint64_t)num_blocks};
+    cuuint64_t strides[3] = {(cuuint64_t)mla::kDQK * 2, 128, (cuuint64_t)mla::kDQK * 2 * mla::kBlockSize};
+    cuuint32_t box[4] = {64, 64, 2, 1};
+    if (!encode(&tm_kv2, kv_cache, 4, dims, strides, box)) return MLA_ERR_INVALID_ARG;
   }
   {
     cuuint64_t dims[2] = {(cuuint64_t)mla::kDLatent, (cuuint64_t)rows};
@@ -226,7 +236,7 @@ mla_status_t launch_attention(const void* q_nope, const void* q_pe, const void* 
   }
   float* part_o = static_cast<float*>(workspace);
   float* part_lse = part_o + g.slots * g.M * mla::kDLatent;
-  if (mla::launch_decode(tm_kv, tm_qn, tm_qp, block_table, max_blocks, cache_seqlens,
+  if (mla::launch_decode(kv_cache, tm_kv, tm_kv2, tm_qn, tm_qp, block_table, max_blocks, cache_seqlens,
                          static_cast<const int32_t*>(metadata), num_blocks, B, s_q, H, softmax_scale, causal != 0,
                          out, lse, part_o, part_lse, status, 2 * g.P * g.T, s) != cudaSuccess)
     return MLA_ERR_CUDA;

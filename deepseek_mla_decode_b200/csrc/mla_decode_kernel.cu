@@ -60,7 +60,8 @@ constexpr uint32_t kIdescPV = make_idesc_bf16(128, 256, false, true);
 constexpr int kBarSoftmax = 1;  // named barrier id for the 256 softmax threads
 
 struct Params {
-  CUtensorMap tm_kv;  // [num_blocks][64][576] bf16, box {64, 64, 1}, SW128
+  CUtensorMap tm_kv;   // [num_blocks][64][576] bf16, box {64, 64, 1}, SW128
+  CUtensorMap tm_kv2;  // same memory as [num_blocks][9][64][64], box {64, 64, 2, 1}, SW128
   CUtensorMap tm_qn;  // [B*M][512] bf16, box {64, 64}, SW128
   CUtensorMap tm_qp;  // [B*M][64] bf16, box {64, 64}, SW128
   const int32_t* block_table;
@@ -160,6 +161,10 @@ __device__ __forceinline__ void set_status(const Params& p, int bits) {
 }
 
 // Bounded wait that also gives up when another role of this CTA aborted.
+// cluster_scope selects acquire.cluster, needed only where the peer CTA's generic
+// shared-memory writes (P, zeroed tail rows) or TMEM reads are published by a
+// release.cluster arrive; data landed by TMA is ordered by its transaction bytes and
+// a CTA-scope wait suffices (the cluster-scope acquire costs ~0.4 us per wait).
 __device__ __forceinline__ bool wait_bar(Ctrl* c, const Params& p, uint32_t bar, uint32_t parity,
                                          bool cluster_scope) {
   const bool ok0 = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
@@ -186,6 +191,22 @@ __device__ __forceinline__ void tma_load_3d_cg2(uint32_t dst, const void* tmap, 
       "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d_cg2(uint32_t dst, const void* tmap, uint32_t bar_cluster,
+                                                int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1,
+                                            int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
 __device__ __forceinline__ void tma_load_2d_cg2(uint32_t dst, const void* tmap, uint32_t bar_cluster,
@@ -286,6 +307,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&p.tm_kv);
+    prefetch_tmap(&p.tm_kv2);
     prefetch_tmap(&p.tm_qn);
     prefetch_tmap(&p.tm_qp);
   }
@@ -411,16 +433,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
               const int d0 = 256 * h + 128 * (int)rank;
               const uint32_t fb = smem_u32(&ctrl.full[slot]);
               if (!needs_tail) {
-                if (lane == 0 && leader) mbar_arrive_expect_tx(fb, 2 * kStageBytes);
-                if (lane < 2)
-                  tma_load_3d_cg2(dst + lane * kChunkBytes, &p.tm_kv, mapa_shared(fb, 0), d0 + 64 * lane, 0, id);
+                if (lane == 0) {
+                  if (leader) mbar_arrive_expect_tx(fb, 2 * kStageBytes);
+                  tma_load_4d_cg2(dst, &p.tm_kv2, mapa_shared(fb, 0), 0, 0, d0 / 64, id);
+                }
               } else {
                 // Land locally, zero rows [rv, 64) of both boxes (NaN-safe: those rows
                 // meet P = 0 inside the last MMA step), then release to the leader.
                 if (lane == 0) {
                   mbar_arrive_expect_tx(tb, kStageBytes);
-                  tma_load_3d(dst, &p.tm_kv, tb, d0, 0, id);
-                  tma_load_3d(dst + kChunkBytes, &p.tm_kv, tb, d0 + 64, 0, id);
+                  tma_load_4d(dst, &p.tm_kv2, tb, 0, 0, d0 / 64, id);
                   ok = wait_bar(&ctrl, p, tb, tail_uses & 1, false);
                 }
                 ++tail_uses;
@@ -466,7 +488,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
       bool ok = true;
       const bool elected = elect_one();
       while (ok && walk.next(pc)) {
-        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.q_full), npieces & 1, true);
+        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.q_full), npieces & 1, false);
         tc_fence_after();
         const int nt = num_tiles(pc);
         auto mma_qk = [&](int t) {
@@ -474,7 +496,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           const uint32_t d = tmem + kTmemS0 + 128 * buf;
           for (int c = 0; c < kQChunks && ok; ++c) {
             const uint32_t slot = it % kStages;
-            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), (it / kStages) & 1, true);
+            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), (it / kStages) & 1, false);
             if (!ok) break;
             tc_fence_after();
             if (elected) {
@@ -506,7 +528,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           for (int h = 0; h < 2 && ok; ++h) {
             for (int kb = 0; kb < nb && ok; ++kb) {
               const uint32_t slot = it % kStages;
-              ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), (it / kStages) & 1, true);
+              ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), (it / kStages) & 1, false);
               const int rv = rows_in_block(pc, t, kb);
               if (ok && (rv & 15) != 0) {  // tail stage: the peer zeroes its copy too
                 ok = wait_bar(&ctrl, p, smem_u32(&ctrl.peer_tail[slot]), (tail_par >> slot) & 1, true);
@@ -769,15 +791,18 @@ cudaError_t decode_kernel_setup(int device) {
   return cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDyn + 1024);
 }
 
-cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
+cudaError_t launch_decode(const void* kv_base, const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
+                          const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
                           const int32_t* block_table, int max_blocks, const int32_t* seqlens,
                           const int32_t* meta, int64_t num_blocks, int B, int s_q, int H, float scale,
                           int causal, void* out, float* lse, float* part_o, float* part_lse,
                           int32_t* status, int num_ctas, cudaStream_t stream) {
   Params prm;
   prm.tm_kv = tm_kv;
+  prm.tm_kv2 = tm_kv2;
   prm.tm_qn = tm_qn;
   prm.tm_qp = tm_qp;
+  (void)kv_base;
   prm.block_table = block_table;
   prm.seqlens = seqlens;
   prm.meta = meta;
