@@ -16,7 +16,7 @@ cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, int max_
                            const float* part_o, const float* part_lse, void* out, float* lse,
                            int32_t* status, cudaStream_t stream);
 cudaError_t decode_kernel_setup(int device);
-cudaError_t launch_decode(const void* kv_base, const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
+cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
                           const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
                           const int32_t* block_table, int max_blocks, const int32_t* seqlens,
                           const int32_t* meta, int64_t num_blocks, int B, int s_q, int H, float scale,
@@ -236,7 +236,7 @@ mla_status_t launch_attention(const void* q_nope, const void* q_pe, const void* 
   }
   float* part_o = static_cast<float*>(workspace);
   float* part_lse = part_o + g.slots * g.M * mla::kDLatent;
-  if (mla::launch_decode(kv_cache, tm_kv, tm_kv2, tm_qn, tm_qp, block_table, max_blocks, cache_seqlens,
+  if (mla::launch_decode(tm_kv, tm_kv2, tm_qn, tm_qp, block_table, max_blocks, cache_seqlens,
                          static_cast<const int32_t*>(metadata), num_blocks, B, s_q, H, softmax_scale, causal != 0,
                          out, lse, part_o, part_lse, status, 2 * g.P * g.T, s) != cudaSuccess)
     return MLA_ERR_CUDA;

@@ -791,7 +791,7 @@ cudaError_t decode_kernel_setup(int device) {
   return cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDyn + 1024);
 }
 
-cudaError_t launch_decode(const void* kv_base, const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
+cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
                           const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
                           const int32_t* block_table, int max_blocks, const int32_t* seqlens,
                           const int32_t* meta, int64_t num_blocks, int B, int s_q, int H, float scale,
@@ -802,7 +802,6 @@ cudaError_t launch_decode(const void* kv_base, const CUtensorMap& tm_kv, const C
   prm.tm_kv2 = tm_kv2;
   prm.tm_qn = tm_qn;
   prm.tm_qp = tm_qp;
-  (void)kv_base;
   prm.block_table = block_table;
   prm.seqlens = seqlens;
   prm.meta = meta;
