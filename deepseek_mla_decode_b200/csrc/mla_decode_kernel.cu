@@ -19,9 +19,10 @@
 //       all 256 dims of that half.
 // O uses TMEM columns [0, 256), the two S buffers [256, 384) and [384, 512).
 //
-// Warp roles (384 threads): warps 0, 2, 3 = TMA producers (alternate ring stages),
+// Warp roles (416 threads): warps 0, 2, 3 = TMA producers (alternate ring stages),
 // warp 1 = MMA issuer (leader CTA only) and TMEM owner, warps 4..11 = softmax /
-// correction / epilogue (thread = one row x 64 keys of S, one row x 128 dims of O).
+// correction / epilogue (thread = one row x 64 keys of S, one row x 128 dims of O),
+// warp 12 = Q loader.
 // Every mbarrier wait is bounded; a
 // timeout sets MLA_DEVICE_ERR_TIMEOUT, raises a CTA-wide abort flag and the kernel
 // drains and returns.
@@ -38,10 +39,11 @@ using namespace ptx;
 
 namespace {
 
-constexpr int kNumThreads = 384;
+constexpr int kNumThreads = 416;
 constexpr int kNumProducers = 3;  // warps 0, 2, 3
 constexpr int kMmaWarp = 1;
-constexpr int kSoftmaxWarp0 = 4;
+constexpr int kSoftmaxWarp0 = 4;   // warps 4..11
+constexpr int kQWarp = 12;
 constexpr int kNumSoftmaxThreads = 256;
 constexpr int kStages = 7;
 constexpr int kStageBytes = 16384;
@@ -89,15 +91,13 @@ struct __align__(8) Ctrl {
   uint64_t p_full;          // leader: P written in both CTAs (count 2)
   uint64_t p_free;          // both: PV done (commit)
   uint64_t o_free;          // leader: O read out by both CTAs (count 2)
-  uint64_t tail[3];         // both: per-producer landing barrier of a stage that needs tail zeroing
-  uint64_t peer_tail[kStages];  // leader: the peer zeroed its copy of the tail stage in this slot
   uint32_t tmem_base;
   volatile int abort;
   float red_max[2][4][64];
   float red_sum[4][64];   // sum of the bf16-rounded weights (normalises the output)
   float red_sum32[4][64]; // sum of the fp32 weights (gives the lse)
   int bad_piece;
-  int block_ids[3][128];  // each producer's window of the current piece's physical block ids
+  int block_ids[3][128];  // each producer's window of physical block ids (current and previous piece)
 };
 constexpr int kIdRing = 128;
 
@@ -162,7 +162,7 @@ __device__ __forceinline__ void set_status(const Params& p, int bits) {
 
 // Bounded wait that also gives up when another role of this CTA aborted.
 // cluster_scope selects acquire.cluster, needed only where the peer CTA's generic
-// shared-memory writes (P, zeroed tail rows) or TMEM reads are published by a
+// shared-memory writes (P) or TMEM reads are published by a
 // release.cluster arrive; data landed by TMA is ordered by its transaction bytes and
 // a CTA-scope wait suffices (the cluster-scope acquire costs ~0.4 us per wait).
 __device__ __forceinline__ bool wait_bar(Ctrl* c, const Params& p, uint32_t bar, uint32_t parity,
@@ -199,14 +199,6 @@ __device__ __forceinline__ void tma_load_4d_cg2(uint32_t dst, const void* tmap, 
       "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1,
-                                            int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
 __device__ __forceinline__ void tma_load_2d_cg2(uint32_t dst, const void* tmap, uint32_t bar_cluster,
@@ -293,8 +285,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     mbar_init(smem_u32(&ctrl.p_full), 2);
     mbar_init(smem_u32(&ctrl.p_free), 1);
     mbar_init(smem_u32(&ctrl.o_free), 2);
-    for (int i = 0; i < 3; ++i) mbar_init(smem_u32(&ctrl.tail[i]), 1);
-    for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&ctrl.peer_tail[s]), 1);
     ctrl.abort = 0;
     fence_mbar_init();
   }
@@ -326,13 +316,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     if (warp == 0 || warp == 2 || warp == 3) {
       const int pi = (warp == 0) ? 0 : warp - 1;
       int32_t* idwin = ctrl.block_ids[pi];
-      const uint32_t tb = smem_u32(&ctrl.tail[pi]);
       PieceWalker walk(p, part);
-      Piece pc;
-      uint32_t it = 0, tail_uses = 0;
-      int npieces = 0;
+      uint32_t it = 0;
       bool ok = true;
-      const uint32_t q_full_l = mapa_shared(smem_u32(&ctrl.q_full), 0);
       auto mine = [&]() { return (int)(it % kNumProducers) == pi; };
       // acquire the ring slot of stage `it` (lane 0)
       auto acquire = [&](uint32_t& slot) -> bool {
@@ -341,140 +327,127 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         if (use > 0 && !wait_bar(&ctrl, p, smem_u32(&ctrl.empty[slot]), (use - 1) & 1, false)) return false;
         return true;
       };
-      while (ok && walk.next(pc)) {
-        const int64_t row_base = (int64_t)pc.b * p.M + tile_row0 + kRowsPerCta * (int)rank;
-        // ---- Q of this piece ----
-        if (pi == 0 && lane == 0) {
-          if (npieces > 0) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.q_empty), (npieces - 1) & 1, false);
-          if (ok) {
-            if (leader) mbar_arrive_expect_tx(smem_u32(&ctrl.q_full), 2 * kQBytes);
-            for (int c = 0; c < kQChunks; ++c) {
-              if (c < 8)
-                tma_load_2d_cg2(sQ + c * kChunkBytes, &p.tm_qn, q_full_l, 64 * c, (int)row_base);
-              else
-                tma_load_2d_cg2(sQ + c * kChunkBytes, &p.tm_qp, q_full_l, 0, (int)row_base);
-            }
-          }
+      // Physical block ids of the current piece, fetched 32 at a time (one coalesced
+      // load per lane) one chunk ahead of use into this warp's 128-entry window, from
+      // window offset `cur_base` on; invalid ids are clamped to block 0 here (the
+      // epilogue turns that piece's rows into NaN).
+      Piece cur{};
+      int cur_base = 0, id_pending = 0, id_chunks = 0;
+      const int32_t* bt = nullptr;
+      auto fetch_id = [&](int i) -> int {
+        return (i < cur.k_hi - cur.k_lo) ? clamp_block_id(p, bt[cur.k_lo + i]) : 0;
+      };
+      auto ensure_ids = [&](int last) {  // make relative blocks <= last of `cur` readable
+        while (last >= 32 * id_chunks) {
+          idwin[(cur_base + 32 * id_chunks + lane) % kIdRing] = id_pending;
+          ++id_chunks;
+          id_pending = fetch_id(32 * id_chunks + lane);
+          __syncwarp();
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        ++npieces;
-        const int nt = num_tiles(pc);
-        const int32_t* bt = p.block_table + (int64_t)pc.b * p.max_blocks;
-        // Physical block ids of the piece, fetched 32 at a time (one coalesced load per
-        // lane) one chunk ahead of use into this warp's 128-entry window; invalid ids
-        // are clamped to block 0 here (the epilogue turns that piece's rows into NaN).
-        const int piece_blocks = pc.k_hi - pc.k_lo;
-        auto fetch_id = [&](int i) -> int {
-          return (i < piece_blocks) ? clamp_block_id(p, bt[pc.k_lo + i]) : 0;
-        };
-        int id_pending = fetch_id(lane);
-        int id_chunks = 0;  // chunks of 32 ids stored in the window
-        auto ensure_ids = [&](int last) {  // make relative blocks <= last readable
-          while (last >= 32 * id_chunks) {
-            idwin[(32 * id_chunks + lane) % kIdRing] = id_pending;
-            ++id_chunks;
-            id_pending = fetch_id(32 * id_chunks + lane);
-            __syncwarp();
+      };
+      auto issue_qk = [&](int t) {
+        const int nb = blocks_in_tile(cur, t);
+        const int own0 = 2 * (int)rank;
+        ensure_ids(t * kBlocksPerTile + nb - 1);
+        // this lane's box (lanes 0 and 1 each issue one of the CTA's two blocks)
+        const int own = min(max(nb - own0, 0), 2);
+        int my_id = idwin[(cur_base + t * kBlocksPerTile + own0 + (lane & 1)) % kIdRing];
+        // Every stage must carry bytes from both CTAs: the leader's full barrier then
+        // cannot complete before the peer has issued the stage, which keeps the peer
+        // producers within one ring cycle of the MMAs (otherwise its empty-barrier
+        // parity could alias).  A peer without keys in this tile loads a copy of the
+        // tile's first block; those S columns are masked.
+        const int nbox = own > 0 ? own : 1;
+        if (own == 0) my_id = idwin[(cur_base + t * kBlocksPerTile) % kIdRing];
+        const int peer_boxes = nb > 2 ? nb - 2 : 1;
+        const int lead_boxes = nb < 2 ? nb : 2;
+        for (int c = 0; c < kQChunks && ok; ++c) {
+          if (!mine()) {
+            ++it;
+            continue;
           }
-        };
-        auto issue_qk = [&](int t) {
-          const int nb = blocks_in_tile(pc, t);
-          const int own0 = 2 * (int)rank;
-          ensure_ids(t * kBlocksPerTile + nb - 1);
-          int ids[2];
-          int own = 0;
-          for (int i = 0; i < 2; ++i)
-            if (own0 + i < nb) ids[own++] = idwin[(t * kBlocksPerTile + own0 + i) % kIdRing];
-          // Every stage must carry bytes from both CTAs: the leader's full barrier then
-          // cannot complete before the peer has issued the stage, which keeps the peer
-          // producers within one ring cycle of the MMAs (otherwise its empty-barrier
-          // parity could alias).  A peer without keys in this tile loads a copy of the
-          // tile's first block; those S columns are masked.
-          if (own == 0) ids[own++] = idwin[(t * kBlocksPerTile) % kIdRing];
-          const int peer_boxes = nb > 2 ? nb - 2 : 1;
-          const int lead_boxes = nb < 2 ? nb : 2;
-          for (int c = 0; c < kQChunks && ok; ++c) {
+          uint32_t slot;
+          if (lane == 0) ok = acquire(slot);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          slot = __shfl_sync(0xffffffffu, slot, 0);
+          // Only the leader arrives (posting both CTAs' bytes); the peer's TMA
+          // completes its bytes on the leader's barrier.
+          const uint32_t fb = smem_u32(&ctrl.full[slot]);
+          if (lane == 0 && leader) mbar_arrive_expect_tx(fb, kChunkBytes * (lead_boxes + peer_boxes));
+          if (lane < nbox)
+            tma_load_3d_cg2(sRing + slot * kStageBytes + lane * kChunkBytes, &p.tm_kv, mapa_shared(fb, 0), 64 * c,
+                            0, my_id);
+          ++it;
+        }
+      };
+      // V stages of tile t of piece pc (ids at window offset base).  The sequence's
+      // last block, with rv < 64 valid keys, is loaded from row rv - 64: the box's
+      // first 64 - rv rows fall before the block and are zero-filled by the TMA, the
+      // keys land in rows [64 - rv, 64).  No row past the sequence end is read, so
+      // the stage needs no zeroing; P of that block is stored shifted to match.
+      auto issue_pv = [&](const Piece& pc, int base, int t) {
+        const int nb = blocks_in_tile(pc, t);
+        for (int h = 0; h < 2 && ok; ++h) {
+          for (int kb = 0; kb < nb && ok; ++kb) {
             if (!mine()) {
               ++it;
               continue;
             }
+            const int id = idwin[(base + t * kBlocksPerTile + kb) % kIdRing];
+            const int rv = rows_in_block(pc, t, kb);
             uint32_t slot;
             if (lane == 0) ok = acquire(slot);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             slot = __shfl_sync(0xffffffffu, slot, 0);
-            // Only the leader arrives (posting both CTAs' bytes); the peer's TMA
-            // completes its bytes on the leader's barrier.
+            const int d0 = 256 * h + 128 * (int)rank;
             const uint32_t fb = smem_u32(&ctrl.full[slot]);
-            if (lane == 0 && leader) mbar_arrive_expect_tx(fb, kChunkBytes * (lead_boxes + peer_boxes));
-            if (lane < own)
-              tma_load_3d_cg2(sRing + slot * kStageBytes + lane * kChunkBytes, &p.tm_kv, mapa_shared(fb, 0), 64 * c,
-                              0, ids[lane]);
+            if (lane == 0) {
+              if (leader) mbar_arrive_expect_tx(fb, 2 * kStageBytes);
+              tma_load_4d_cg2(sRing + slot * kStageBytes, &p.tm_kv2, mapa_shared(fb, 0), 0, rv - kBlockSize, d0 / 64,
+                              id);
+            }
             ++it;
           }
-        };
-        auto issue_pv = [&](int t) {
-          const int nb = blocks_in_tile(pc, t);
-          for (int h = 0; h < 2 && ok; ++h) {
-            for (int kb = 0; kb < nb && ok; ++kb) {
-              if (!mine()) {
-                ++it;
-                continue;
-              }
-              const int id = idwin[(t * kBlocksPerTile + kb) % kIdRing];
-              const int rv = rows_in_block(pc, t, kb);
-              const bool needs_tail = (rv & 15) != 0;  // a partial 16-key MMA step reads rows >= n
-              uint32_t slot;
-              if (lane == 0) ok = acquire(slot);
-              ok = __shfl_sync(0xffffffffu, ok, 0);
-              if (!ok) break;
-              slot = __shfl_sync(0xffffffffu, slot, 0);
-              const uint32_t dst = sRing + slot * kStageBytes;
-              const int d0 = 256 * h + 128 * (int)rank;
-              const uint32_t fb = smem_u32(&ctrl.full[slot]);
-              if (!needs_tail) {
-                if (lane == 0) {
-                  if (leader) mbar_arrive_expect_tx(fb, 2 * kStageBytes);
-                  tma_load_4d_cg2(dst, &p.tm_kv2, mapa_shared(fb, 0), 0, 0, d0 / 64, id);
-                }
-              } else {
-                // Land locally, zero rows [rv, 64) of both boxes (NaN-safe: those rows
-                // meet P = 0 inside the last MMA step), then release to the leader.
-                if (lane == 0) {
-                  mbar_arrive_expect_tx(tb, kStageBytes);
-                  tma_load_4d(dst, &p.tm_kv2, tb, 0, 0, d0 / 64, id);
-                  ok = wait_bar(&ctrl, p, tb, tail_uses & 1, false);
-                }
-                ++tail_uses;
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (ok) {
-                  // 2 boxes x (64 - rv) rows x 128 B, 16 B per store
-                  const int nvec = 2 * (kBlockSize - rv) * 8;
-                  for (int v = lane; v < nvec; v += 32) {
-                    const int box = v / ((kBlockSize - rv) * 8);
-                    const int rem = v % ((kBlockSize - rv) * 8);
-                    const uint32_t a = dst + box * kChunkBytes + (rv + rem / 8) * 128 + (rem % 8) * 16;
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
-                  }
-                  fence_proxy_async_smem();
-                  __syncwarp();
-                  if (lane == 0) {
-                    if (leader)
-                      mbar_arrive(fb);  // the stage's only arrival, no bytes
-                    else
-                      mbar_arrive_remote(mapa_shared(smem_u32(&ctrl.peer_tail[slot]), 0));
-                  }
-                }
-              }
-              ++it;
-            }
-          }
-        };
+        }
+      };
+      // Ring order per piece: QK(0), then QK(t) followed by PV(t - 1), then PV(last).
+      while (ok && walk.next(cur)) {
+        bt = p.block_table + (int64_t)cur.b * p.max_blocks;
+        id_chunks = 0;
+        id_pending = fetch_id(lane);
+        const int nt = num_tiles(cur);
         for (int t = 0; t < nt && ok; ++t) {
           issue_qk(t);
-          if (t >= 1) issue_pv(t - 1);
+          if (t >= 1 && ok) issue_pv(cur, cur_base, t - 1);
         }
-        if (ok) issue_pv(nt - 1);
+        if (ok) issue_pv(cur, cur_base, nt - 1);
+        cur_base = (cur_base + 32 * id_chunks) % kIdRing;
+      }
+    }
+    // =======================================================================
+    // Q loader (both CTAs): Q of piece k + 1 is loaded as soon as the last QK of
+    // piece k has completed, while the MMAs still work through the PV of piece k.
+    // =======================================================================
+    else if (warp == kQWarp) {
+      if (lane == 0) {
+        PieceWalker walk(p, part);
+        Piece pc;
+        int npieces = 0;
+        const uint32_t q_full_l = mapa_shared(smem_u32(&ctrl.q_full), 0);
+        while (walk.next(pc)) {
+          if (npieces > 0 && !wait_bar(&ctrl, p, smem_u32(&ctrl.q_empty), (npieces - 1) & 1, false)) break;
+          const int row_base = pc.b * p.M + tile_row0 + kRowsPerCta * (int)rank;
+          if (leader) mbar_arrive_expect_tx(smem_u32(&ctrl.q_full), 2 * kQBytes);
+          for (int c = 0; c < kQChunks; ++c) {
+            if (c < 8)
+              tma_load_2d_cg2(sQ + c * kChunkBytes, &p.tm_qn, q_full_l, 64 * c, row_base);
+            else
+              tma_load_2d_cg2(sQ + c * kChunkBytes, &p.tm_qp, q_full_l, 0, row_base);
+          }
+          ++npieces;
+        }
       }
     }
     // =======================================================================
@@ -482,89 +455,88 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     // =======================================================================
     else if (warp == kMmaWarp && leader) {
       PieceWalker walk(p, part);
-      Piece pc;
-      uint32_t it = 0, qk_count = 0, pv_count = 0, tail_par = 0;
+      uint32_t it = 0, qk_count = 0, pv_count = 0;
       int npieces = 0;
       bool ok = true;
       const bool elected = elect_one();
-      while (ok && walk.next(pc)) {
-        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.q_full), npieces & 1, false);
+      auto mma_qk = [&](int nt, int t) {
+        const uint32_t buf = qk_count & 1;
+        const uint32_t d = tmem + kTmemS0 + 128 * buf;
+        for (int c = 0; c < kQChunks && ok; ++c) {
+          const uint32_t slot = it % kStages;
+          ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), (it / kStages) & 1, false);
+          if (!ok) break;
+          tc_fence_after();
+          if (elected) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t a = make_smem_desc(sQ + c * kChunkBytes + ks * 32, 16, 1024, kSwizzle128B);
+              const uint64_t b = make_smem_desc(sRing + slot * kStageBytes + ks * 32, 16, 1024, kSwizzle128B);
+              umma_2sm(d, a, b, kIdescQK, (c | ks) != 0);
+            }
+            commit_2sm(smem_u32(&ctrl.empty[slot]));
+          }
+          __syncwarp();
+          ++it;
+        }
+        if (elected && ok) {
+          commit_2sm(smem_u32(&ctrl.s_full[buf]));
+          if (t == nt - 1) commit_2sm(smem_u32(&ctrl.q_empty));
+        }
+        __syncwarp();
+        ++qk_count;
+      };
+      // PV of tile t of piece pc, the piece_idx-th piece of this partition
+      auto mma_pv = [&](const Piece& pc, int piece_idx, int t) {
+        if (!ok) return;
+        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_full), pv_count & 1, true);
+        if (ok && t == 0 && piece_idx > 0) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.o_free), (piece_idx - 1) & 1, true);
+        if (!ok) return;
         tc_fence_after();
-        const int nt = num_tiles(pc);
-        auto mma_qk = [&](int t) {
-          const uint32_t buf = qk_count & 1;
-          const uint32_t d = tmem + kTmemS0 + 128 * buf;
-          for (int c = 0; c < kQChunks && ok; ++c) {
+        const int nb = blocks_in_tile(pc, t);
+        for (int h = 0; h < 2 && ok; ++h) {
+          for (int kb = 0; kb < nb && ok; ++kb) {
             const uint32_t slot = it % kStages;
             ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), (it / kStages) & 1, false);
             if (!ok) break;
             tc_fence_after();
+            // the sequence's last block sits in rows [64 - rv, 64): skip whole zero steps
+            const int rv = rows_in_block(pc, t, kb);
+            const int ks0 = (kBlockSize - rv) >> 4;
             if (elected) {
-#pragma unroll
-              for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t a = make_smem_desc(sQ + c * kChunkBytes + ks * 32, 16, 1024, kSwizzle128B);
-                const uint64_t b = make_smem_desc(sRing + slot * kStageBytes + ks * 32, 16, 1024, kSwizzle128B);
-                umma_2sm(d, a, b, kIdescQK, (c | ks) != 0);
+              for (int ks = ks0; ks < 4; ++ks) {
+                const uint64_t a = make_smem_desc(sP + kb * kChunkBytes + ks * 32, 16, 1024, kSwizzle128B);
+                const uint64_t b = make_smem_desc(sRing + slot * kStageBytes + ks * 2048, 8192, 1024, kSwizzle128B);
+                umma_2sm(tmem + kTmemO + 128 * h, a, b, kIdescPV, !(t == 0 && kb == 0 && ks == ks0));
               }
               commit_2sm(smem_u32(&ctrl.empty[slot]));
             }
             __syncwarp();
             ++it;
           }
-          if (elected && ok) {
-            commit_2sm(smem_u32(&ctrl.s_full[buf]));
-            if (t == nt - 1) commit_2sm(smem_u32(&ctrl.q_empty));
-          }
-          __syncwarp();
-          ++qk_count;
-        };
-        auto mma_pv = [&](int t) {
-          if (!ok) return;
-          ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_full), pv_count & 1, true);
-          if (ok && t == 0 && npieces > 0) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.o_free), (npieces - 1) & 1, true);
-          if (!ok) return;
-          tc_fence_after();
-          const int nb = blocks_in_tile(pc, t);
-          for (int h = 0; h < 2 && ok; ++h) {
-            for (int kb = 0; kb < nb && ok; ++kb) {
-              const uint32_t slot = it % kStages;
-              ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), (it / kStages) & 1, false);
-              const int rv = rows_in_block(pc, t, kb);
-              if (ok && (rv & 15) != 0) {  // tail stage: the peer zeroes its copy too
-                ok = wait_bar(&ctrl, p, smem_u32(&ctrl.peer_tail[slot]), (tail_par >> slot) & 1, true);
-                tail_par ^= 1u << slot;
-              }
-              if (!ok) break;
-              tc_fence_after();
-              const int ksteps = (rv + 15) >> 4;
-              if (elected) {
-                for (int ks = 0; ks < ksteps; ++ks) {
-                  const uint64_t a = make_smem_desc(sP + kb * kChunkBytes + ks * 32, 16, 1024, kSwizzle128B);
-                  const uint64_t b = make_smem_desc(sRing + slot * kStageBytes + ks * 2048, 8192, 1024, kSwizzle128B);
-                  umma_2sm(tmem + kTmemO + 128 * h, a, b, kIdescPV, !(t == 0 && kb == 0 && ks == 0));
-                }
-                commit_2sm(smem_u32(&ctrl.empty[slot]));
-              }
-              __syncwarp();
-              ++it;
-            }
-          }
-          if (elected && ok) commit_2sm(smem_u32(&ctrl.p_free));
-          __syncwarp();
-          ++pv_count;
-        };
-        for (int t = 0; t < nt && ok; ++t) {
-          mma_qk(t);
-          if (t >= 1) mma_pv(t - 1);
         }
-        mma_pv(nt - 1);
+        if (elected && ok) commit_2sm(smem_u32(&ctrl.p_free));
+        __syncwarp();
+        ++pv_count;
+      };
+      // same ring order as the producers
+      Piece cur;
+      while (ok && walk.next(cur)) {
+        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.q_full), npieces & 1, false);
+        tc_fence_after();
+        const int nt = num_tiles(cur);
+        for (int t = 0; t < nt && ok; ++t) {
+          mma_qk(nt, t);
+          if (t >= 1) mma_pv(cur, npieces, t - 1);
+        }
+        mma_pv(cur, npieces, nt - 1);
         ++npieces;
       }
     }
     // =======================================================================
     // softmax / correction / epilogue
     // =======================================================================
-    else if (warp >= kSoftmaxWarp0) {
+    else if (warp >= kSoftmaxWarp0 && warp < kSoftmaxWarp0 + 8) {
       const int st = tid - kSoftmaxWarp0 * 32;  // 0..255
       const int g = st >> 7;                   // column group: keys 64g.. of each half; O half g
       const int L = st & 127;                  // TMEM lane
@@ -679,6 +651,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
                     : "memory");
               }
               tmem_wait_st();
+            }
+          }
+          // The sequence's last block (rv < 64 keys) was loaded into rows [64 - rv, 64)
+          // of its V stage: shift its P row right by 64 - rv keys to match (the keys
+          // shifted out are >= rv, whose weights are 0; zeros are shifted in).
+          {
+            const int rv = pc.n - key0;
+            if (rv > 0 && rv < kBlockSize) {  // warp-uniform: the warp's rows share the block
+              const int sh = kBlockSize - rv;
+              if (sh & 1) {
+#pragma unroll
+                for (int w = 31; w >= 1; --w) pk[w] = __byte_perm(pk[w - 1], pk[w], 0x5432);
+                pk[0] <<= 16;
+              }
+              const int ws = sh >> 1;
+#pragma unroll
+              for (int bit = 0; bit < 5; ++bit) {
+                if ((ws >> bit) & 1) {
+#pragma unroll
+                  for (int w = 31; w >= 0; --w) pk[w] = (w >= (1 << bit)) ? pk[w - (1 << bit)] : 0u;
+                }
+              }
             }
           }
           // P -> shared memory: chunk (2 hk + g) holds keys 64 (2hk+g) .. of all 64 rows,
