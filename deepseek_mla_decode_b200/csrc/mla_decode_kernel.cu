@@ -185,22 +185,6 @@ __device__ __forceinline__ bool wait_bar(Ctrl* c, const Params& p, uint32_t bar,
   }
 }
 
-__device__ __forceinline__ void tma_load_3d_cg2(uint32_t dst, const void* tmap, uint32_t bar_cluster,
-                                                int c0, int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_4d_cg2(uint32_t dst, const void* tmap, uint32_t bar_cluster,
-                                                int c0, int c1, int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
 __device__ __forceinline__ void tma_load_2d_cg2(uint32_t dst, const void* tmap, uint32_t bar_cluster,
                                                 int c0, int c1) {
   asm volatile(
@@ -209,18 +193,48 @@ __device__ __forceinline__ void tma_load_2d_cg2(uint32_t dst, const void* tmap, 
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1)
       : "memory");
 }
-__device__ __forceinline__ void umma_2sm(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+// Predicated forms: the whole warp executes the instruction and only lanes with
+// `on` set issue it, so the issuing warp never diverges around the issue.
+__device__ __forceinline__ void umma_2sm_if(bool on, uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                            uint32_t acc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+      "@q tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"((uint32_t)on)
       : "memory");
 }
-__device__ __forceinline__ void commit_2sm(uint32_t bar) {
+__device__ __forceinline__ void commit_2sm_if(bool on, uint32_t bar) {
   asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(bar),
-      "h"((uint16_t)0x3)
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
+      "@q tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %2;\n\t}" ::"r"(bar),
+      "r"((uint32_t)on), "h"((uint16_t)0x3)
+      : "memory");
+}
+__device__ __forceinline__ void expect_tx_if(bool on, uint32_t bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\t"
+      "@q mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(bar),
+      "r"(bytes), "r"((uint32_t)on)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_cg2_if(bool on, uint32_t dst, const void* tmap, uint32_t bar_cluster,
+                                                   int c0, int c1, int c2) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %6, 0;\n\t"
+      "@q cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];\n\t}" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"((uint32_t)on)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d_cg2_if(bool on, uint32_t dst, const void* tmap, uint32_t bar_cluster,
+                                                   int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %7, 0;\n\t"
+      "@q cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];\n\t}" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+      "r"((uint32_t)on)
       : "memory");
 }
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
@@ -320,7 +334,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       auto mine = [&]() { return (int)(it % kNumProducers) == pi; };
-      // acquire the ring slot of stage `it` (lane 0)
+      // acquire the ring slot of stage `it` (every lane waits, the warp stays converged)
       auto acquire = [&](uint32_t& slot) -> bool {
         slot = it % kStages;
         const uint32_t use = it / kStages;
@@ -367,17 +381,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
             continue;
           }
           uint32_t slot;
-          if (lane == 0) ok = acquire(slot);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ok = __shfl_sync(0xffffffffu, acquire(slot), 0);
           if (!ok) break;
-          slot = __shfl_sync(0xffffffffu, slot, 0);
           // Only the leader arrives (posting both CTAs' bytes); the peer's TMA
           // completes its bytes on the leader's barrier.
           const uint32_t fb = smem_u32(&ctrl.full[slot]);
-          if (lane == 0 && leader) mbar_arrive_expect_tx(fb, kChunkBytes * (lead_boxes + peer_boxes));
-          if (lane < nbox)
-            tma_load_3d_cg2(sRing + slot * kStageBytes + lane * kChunkBytes, &p.tm_kv, mapa_shared(fb, 0), 64 * c,
-                            0, my_id);
+          expect_tx_if(lane == 0 && leader, fb, kChunkBytes * (lead_boxes + peer_boxes));
+          tma_load_3d_cg2_if(lane < nbox, sRing + slot * kStageBytes + (lane & 1) * kChunkBytes, &p.tm_kv,
+                             mapa_shared(fb, 0), 64 * c, 0, my_id);
           ++it;
         }
       };
@@ -397,17 +408,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
             const int id = idwin[(base + t * kBlocksPerTile + kb) % kIdRing];
             const int rv = rows_in_block(pc, t, kb);
             uint32_t slot;
-            if (lane == 0) ok = acquire(slot);
-            ok = __shfl_sync(0xffffffffu, ok, 0);
+            ok = __shfl_sync(0xffffffffu, acquire(slot), 0);
             if (!ok) break;
-            slot = __shfl_sync(0xffffffffu, slot, 0);
             const int d0 = 256 * h + 128 * (int)rank;
             const uint32_t fb = smem_u32(&ctrl.full[slot]);
-            if (lane == 0) {
-              if (leader) mbar_arrive_expect_tx(fb, 2 * kStageBytes);
-              tma_load_4d_cg2(sRing + slot * kStageBytes, &p.tm_kv2, mapa_shared(fb, 0), 0, rv - kBlockSize, d0 / 64,
-                              id);
-            }
+            expect_tx_if(lane == 0 && leader, fb, 2 * kStageBytes);
+            tma_load_4d_cg2_if(lane == 0, sRing + slot * kStageBytes, &p.tm_kv2, mapa_shared(fb, 0), 0,
+                               rv - kBlockSize, d0 / 64, id);
             ++it;
           }
         }
@@ -467,23 +474,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), (it / kStages) & 1, false);
           if (!ok) break;
           tc_fence_after();
-          if (elected) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t a = make_smem_desc(sQ + c * kChunkBytes + ks * 32, 16, 1024, kSwizzle128B);
-              const uint64_t b = make_smem_desc(sRing + slot * kStageBytes + ks * 32, 16, 1024, kSwizzle128B);
-              umma_2sm(d, a, b, kIdescQK, (c | ks) != 0);
-            }
-            commit_2sm(smem_u32(&ctrl.empty[slot]));
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t a = make_smem_desc(sQ + c * kChunkBytes + ks * 32, 16, 1024, kSwizzle128B);
+            const uint64_t b = make_smem_desc(sRing + slot * kStageBytes + ks * 32, 16, 1024, kSwizzle128B);
+            umma_2sm_if(elected, d, a, b, kIdescQK, (c | ks) != 0);
           }
-          __syncwarp();
+          commit_2sm_if(elected, smem_u32(&ctrl.empty[slot]));
           ++it;
         }
-        if (elected && ok) {
-          commit_2sm(smem_u32(&ctrl.s_full[buf]));
-          if (t == nt - 1) commit_2sm(smem_u32(&ctrl.q_empty));
+        if (ok) {
+          commit_2sm_if(elected, smem_u32(&ctrl.s_full[buf]));
+          if (t == nt - 1) commit_2sm_if(elected, smem_u32(&ctrl.q_empty));
         }
-        __syncwarp();
         ++qk_count;
       };
       // PV of tile t of piece pc, the piece_idx-th piece of this partition
@@ -503,20 +506,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
             // the sequence's last block sits in rows [64 - rv, 64): skip whole zero steps
             const int rv = rows_in_block(pc, t, kb);
             const int ks0 = (kBlockSize - rv) >> 4;
-            if (elected) {
-              for (int ks = ks0; ks < 4; ++ks) {
-                const uint64_t a = make_smem_desc(sP + kb * kChunkBytes + ks * 32, 16, 1024, kSwizzle128B);
-                const uint64_t b = make_smem_desc(sRing + slot * kStageBytes + ks * 2048, 8192, 1024, kSwizzle128B);
-                umma_2sm(tmem + kTmemO + 128 * h, a, b, kIdescPV, !(t == 0 && kb == 0 && ks == ks0));
-              }
-              commit_2sm(smem_u32(&ctrl.empty[slot]));
+            for (int ks = ks0; ks < 4; ++ks) {
+              const uint64_t a = make_smem_desc(sP + kb * kChunkBytes + ks * 32, 16, 1024, kSwizzle128B);
+              const uint64_t b = make_smem_desc(sRing + slot * kStageBytes + ks * 2048, 8192, 1024, kSwizzle128B);
+              umma_2sm_if(elected, tmem + kTmemO + 128 * h, a, b, kIdescPV, !(t == 0 && kb == 0 && ks == ks0));
             }
-            __syncwarp();
+            commit_2sm_if(elected, smem_u32(&ctrl.empty[slot]));
             ++it;
           }
         }
-        if (elected && ok) commit_2sm(smem_u32(&ctrl.p_free));
-        __syncwarp();
+        if (ok) commit_2sm_if(elected, smem_u32(&ctrl.p_free));
         ++pv_count;
       };
       // same ring order as the producers
