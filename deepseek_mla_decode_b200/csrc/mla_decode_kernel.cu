@@ -462,26 +462,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     // =======================================================================
     else if (warp == kMmaWarp && leader) {
       PieceWalker walk(p, part);
-      uint32_t it = 0, qk_count = 0, pv_count = 0;
+      uint32_t slot = 0, phase = 0, qk_count = 0, pv_count = 0;
       int npieces = 0;
       bool ok = true;
       const bool elected = elect_one();
+      // Shared-memory descriptors: the 14-bit start field holds address >> 4, so the
+      // operand of chunk c / slot s / 16-element K step k is the base plus
+      // c * (8192 >> 4) / s * (16384 >> 4) / k * (32 >> 4) (K-major) or k * (2048 >> 4)
+      // (V, MN-major: 16 keys = 16 rows of 128 bytes).
+      const uint64_t dq0 = make_smem_desc(sQ, 16, 1024, kSwizzle128B);
+      const uint64_t dp0 = make_smem_desc(sP, 16, 1024, kSwizzle128B);
+      const uint64_t dk0 = make_smem_desc(sRing, 16, 1024, kSwizzle128B);
+      const uint64_t dv0 = make_smem_desc(sRing, 8192, 1024, kSwizzle128B);
+      constexpr uint64_t kChunkD = kChunkBytes >> 4, kStageD = kStageBytes >> 4;
+      auto next_stage = [&]() {
+        if (++slot == kStages) {
+          slot = 0;
+          phase ^= 1;
+        }
+      };
       auto mma_qk = [&](int nt, int t) {
         const uint32_t buf = qk_count & 1;
         const uint32_t d = tmem + kTmemS0 + 128 * buf;
         for (int c = 0; c < kQChunks && ok; ++c) {
-          const uint32_t slot = it % kStages;
-          ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), (it / kStages) & 1, false);
+          ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), phase, false);
           if (!ok) break;
           tc_fence_after();
+          const uint64_t a0 = dq0 + c * kChunkD, b0 = dk0 + slot * kStageD;
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t a = make_smem_desc(sQ + c * kChunkBytes + ks * 32, 16, 1024, kSwizzle128B);
-            const uint64_t b = make_smem_desc(sRing + slot * kStageBytes + ks * 32, 16, 1024, kSwizzle128B);
-            umma_2sm_if(elected, d, a, b, kIdescQK, (c | ks) != 0);
-          }
+          for (int ks = 0; ks < 4; ++ks) umma_2sm_if(elected, d, a0 + 2 * ks, b0 + 2 * ks, kIdescQK, (c | ks) != 0);
           commit_2sm_if(elected, smem_u32(&ctrl.empty[slot]));
-          ++it;
+          next_stage();
         }
         if (ok) {
           commit_2sm_if(elected, smem_u32(&ctrl.s_full[buf]));
@@ -499,20 +510,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         const int nb = blocks_in_tile(pc, t);
         for (int h = 0; h < 2 && ok; ++h) {
           for (int kb = 0; kb < nb && ok; ++kb) {
-            const uint32_t slot = it % kStages;
-            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), (it / kStages) & 1, false);
+            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), phase, false);
             if (!ok) break;
             tc_fence_after();
             // the sequence's last block sits in rows [64 - rv, 64): skip whole zero steps
             const int rv = rows_in_block(pc, t, kb);
             const int ks0 = (kBlockSize - rv) >> 4;
-            for (int ks = ks0; ks < 4; ++ks) {
-              const uint64_t a = make_smem_desc(sP + kb * kChunkBytes + ks * 32, 16, 1024, kSwizzle128B);
-              const uint64_t b = make_smem_desc(sRing + slot * kStageBytes + ks * 2048, 8192, 1024, kSwizzle128B);
-              umma_2sm_if(elected, tmem + kTmemO + 128 * h, a, b, kIdescPV, !(t == 0 && kb == 0 && ks == ks0));
-            }
+            const bool first = (t == 0 && kb == 0);
+            const uint64_t a0 = dp0 + kb * kChunkD, b0 = dv0 + slot * kStageD;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              umma_2sm_if(elected && ks >= ks0, tmem + kTmemO + 128 * h, a0 + 2 * ks, b0 + 128 * ks, kIdescPV,
+                          !(first && ks == ks0));
             commit_2sm_if(elected, smem_u32(&ctrl.empty[slot]));
-            ++it;
+            next_stage();
           }
         }
         if (ok) commit_2sm_if(elected, smem_u32(&ctrl.p_free));
