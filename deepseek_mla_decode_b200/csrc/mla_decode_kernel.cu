@@ -572,7 +572,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         // l_part: sum of the bf16 weights that enter the PV MMA (output normaliser, so
         // the weights sum to one exactly); l32_part: fp32 weights (the lse).
         float m_used = -INFINITY, l_part = 0.f, l32_part = 0.f;
-        // Block-id validity of the piece (loads issued now, consumed at the epilogue).
+        // Block-id validity and split layout of the piece (loads issued now, consumed
+        // at the epilogue).
+        const int nsplit = p.meta[off_num_splits(p.B) + pc.b];
+        const int split_base = p.meta[off_split_prefix(p.B) + pc.b];
         int bad_ids = 0;
         {
           const int32_t* bt = p.block_table + (int64_t)pc.b * p.max_blocks;
@@ -710,10 +713,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         }
         if (!ok) break;
         // ---- epilogue of the piece ----------------------------------------
-        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1, false);
-        if (!ok) break;
-        ++pv_count;
-        tc_fence_after();
+        // Row sums and the block-id verdict are final after the last tile's P: reduce
+        // them while the last PV is still running.
         ctrl.red_sum[2 * hk + g][m] = l_part;
         ctrl.red_sum32[2 * hk + g][m] = l32_part;
         if (st == 0) ctrl.bad_piece = 0;
@@ -724,7 +725,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
             ctrl.red_sum32[0][m] + ctrl.red_sum32[1][m] + ctrl.red_sum32[2][m] + ctrl.red_sum32[3][m];
         named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
         const bool bad = ctrl.bad_piece != 0;
-        const int nsplit = p.meta[off_num_splits(p.B) + pc.b];
         const bool direct = (nsplit == 1);
         const float nanf_ = __int_as_float(0x7fc00000);
         const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
@@ -732,29 +732,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
             bad ? nanf_ : ((l32_row > 0.f) ? (m_used + __log2f(l32_row)) * 0.69314718055994531f : -INFINITY);
         const int dim0 = 256 * g + 128 * hk;
         const int64_t orow = (int64_t)pc.b * p.M + grow;
-        const int64_t slot = (int64_t)p.meta[off_split_prefix(p.B) + pc.b] + pc.split;
+        const int64_t slot = (int64_t)split_base + pc.split;
+        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1, false);
+        if (!ok) break;
+        ++pv_count;
+        tc_fence_after();
         const uint32_t to = tmem + kTmemO + 128 * g + lane_off;
-#pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(to + c, o);
-          tmem_wait_ld();
-          if (row_valid) {
-            float v[32];
+        // a bad piece's rows become NaN: scaling by NaN turns every value into NaN
+        const float sc = bad ? nanf_ : inv_l;
+        auto emit = [&](const uint32_t (&o)[32], int c) {
+          if (!row_valid) return;
+          auto v = [&](int j) { return __uint_as_float(o[j]) * sc; };
+          if (direct) {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDLatent + dim0 + c);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = bad ? nanf_ : __uint_as_float(o[j]) * inv_l;
-            if (direct) {
-              uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDLatent + dim0 + c);
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(pack_bf16x2(v(8 * j), v(8 * j + 1)), pack_bf16x2(v(8 * j + 2), v(8 * j + 3)),
+                                  pack_bf16x2(v(8 * j + 4), v(8 * j + 5)), pack_bf16x2(v(8 * j + 6), v(8 * j + 7)));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * p.M + grow) * kDLatent + dim0 + c);
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
-                dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
-                                    pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
-            } else {
-              float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * p.M + grow) * kDLatent + dim0 + c);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            }
+            for (int j = 0; j < 8; ++j) dst[j] = make_float4(v(4 * j), v(4 * j + 1), v(4 * j + 2), v(4 * j + 3));
           }
+        };
+        // two 32-column TMEM loads in flight per wait
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 64) {
+          uint32_t o0[32], o1[32];
+          tmem_ld32(to + c, o0);
+          tmem_ld32(to + c + 32, o1);
+          tmem_wait_ld();
+          emit(o0, c);
+          emit(o1, c + 32);
         }
         if (row_valid && hk == 0 && g == 0) {
           if (direct)
