@@ -14,8 +14,8 @@ constexpr int kTileKeys = 256;     // keys per pipeline step (4 cache blocks)
 constexpr int kBlocksPerTile = kTileKeys / kBlockSize;
 
 // Split-KV scheduler constants (the same values are stated in the float64 oracle).
-constexpr int kSchedOverheadBlocks = 4;  // cost of starting a piece, in blocks
-constexpr int kSchedMinCap = 8;          // smallest partition cost
+constexpr int kSchedOverheadTiles = 1;  // cost of starting a sequence, in 256-key tiles
+constexpr int kSchedMinCap = 2;         // smallest partition cost, in tiles
 constexpr int kMaxWorkers = 256;         // CTA pairs the metadata can describe
 
 // ---------------------------------------------------------------------------

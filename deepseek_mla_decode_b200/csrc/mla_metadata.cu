@@ -2,12 +2,13 @@
 // the decode kernel and the combine kernel follow.  Integer-only; the float64 oracle
 // states the same algorithm and the tests compare the two word for word.
 //
-// Cost model: every 64-row block costs 1 and every sequence with at least one block
-// costs kSchedOverheadBlocks more, placed before its first block.  pre[b] is the cost
-// of the sequences before b, so block k of sequence b sits at position
-// pre[b] + overhead + k.  With P partitions per row tile and
-// cap = max(kSchedMinCap, ceil(total / P)), block (b, k) belongs to partition
-// floor(position / cap): contiguous, near-equal ranges.  (Split-K parallelism is named
+// Cost model, in key tiles of kBlocksPerTile blocks (256 keys): every tile costs 1
+// and every sequence with at least one block costs kSchedOverheadTiles more, placed
+// before its first tile.  pre[b] is the cost of the sequences before b, so tile j of
+// sequence b sits at position pre[b] + overhead + j.  With P partitions per row tile
+// and cap = max(kSchedMinCap, ceil(total / P)), tile (b, j) and its blocks belong to
+// partition floor(position / cap): contiguous, near-equal ranges that are cut only
+// on tile boundaries, so a split adds no ragged tile.  (Split-K parallelism is named
 // in the "DeepSeek speed test / FA3" article, section 2.1; this cost model is ours.)
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -74,7 +75,7 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
       const int n = seqlens[b];
       const int nb = n > 0 ? (n + kBlockSize - 1) / kBlockSize : 0;
       nblk_out[b] = nb;
-      cost = nb > 0 ? nb + kSchedOverheadBlocks : 0;
+      cost = nb > 0 ? (nb + kBlocksPerTile - 1) / kBlocksPerTile + kSchedOverheadTiles : 0;
     }
     int64_t t;
     block_exclusive_scan(cost, scratch, &t);
@@ -99,24 +100,25 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
     if (b < B) {
       const int n = seqlens[b];
       nb = n > 0 ? (n + kBlockSize - 1) / kBlockSize : 0;
-      cost = nb > 0 ? nb + kSchedOverheadBlocks : 0;
+      cost = nb > 0 ? (nb + kBlocksPerTile - 1) / kBlocksPerTile + kSchedOverheadTiles : 0;
     }
     int64_t chunk_total;
     const int64_t pre = s_carry + block_exclusive_scan(cost, scratch, &chunk_total);
     if (b < B) {
       if (nb > 0) {
-        const int64_t first_pos = pre + kSchedOverheadBlocks;
+        const int64_t first_pos = pre + kSchedOverheadTiles;
+        const int64_t nt = (nb + kBlocksPerTile - 1) / kBlocksPerTile;
         const int64_t p0 = first_pos / cap;
-        const int64_t p1 = (first_pos + nb - 1) / cap;
+        const int64_t p1 = (first_pos + nt - 1) / cap;
         first_part[b] = (int32_t)p0;
         num_splits[b] = (int32_t)(p1 - p0 + 1);
         // partitions whose start position falls in [pre, pre + cost)
         const int64_t lo = (pre + cap - 1) / cap;
         const int64_t hi = (pre + cost - 1) / cap;
         for (int64_t p = lo; p <= hi && p < P; ++p) {
-          const int64_t k = p * cap - first_pos;
+          const int64_t j = p * cap - first_pos;  // first tile of partition p
           part_start[2 * p] = b;
-          part_start[2 * p + 1] = (int32_t)(k > 0 ? k : 0);
+          part_start[2 * p + 1] = (int32_t)(j > 0 ? j * kBlocksPerTile : 0);
         }
       } else {
         first_part[b] = 0;
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
     meta[kHdrCap] = (int32_t)cap;
     meta[kHdrTotalSlots] = (int32_t)s_total;
     meta[kHdrNumWorkers] = num_workers;
-    meta[kHdrOverhead] = kSchedOverheadBlocks;
+    meta[kHdrOverhead] = kSchedOverheadTiles;
     for (int i = kHdrOverhead + 1; i < kHdrWords; ++i) meta[i] = 0;
   }
 }

@@ -81,9 +81,10 @@ mla_status_t mla_metadata_size(int B, int s_q, int H, size_t* bytes);
 /*
  * Split-KV schedule for one decode step (shared by every layer of that step).
  *
- * The concatenation of all sequences' 64-row blocks is cut into contiguous ranges of
- * near-equal cost, one per partition; every sequence also costs a fixed overhead
- * before its first block.  A sequence cut across partitions is computed as several
+ * The concatenation of all sequences' key tiles (four 64-row blocks, 256 keys) is cut
+ * into contiguous ranges of near-equal cost, one per partition, only on tile
+ * boundaries; every sequence also costs a fixed overhead of one tile before its
+ * first tile.  A sequence cut across partitions is computed as several
  * partial results that mla_decode merges by log-sum-exp (split-K parallelism, "DeepSeek
  * speed test / FA3" article section 2.1; the cost model is this library's own).
  *

@@ -188,22 +188,26 @@ def lse_combine_ref(o_parts: List[np.ndarray], lse_parts: List[np.ndarray]):
 # ----------------------------------------------------------------------------
 # split-KV schedule (integer; bit-exact target for the device scheduler)
 # ----------------------------------------------------------------------------
-SCHED_OVERHEAD_BLOCKS = 4  # cost of starting a piece, in 64-row blocks
-SCHED_MIN_CAP = 8  # smallest partition cost, so tiny problems are not shattered
+SCHED_KEYS_PER_TILE = 256  # scheduling unit: a key tile of 4 blocks
+SCHED_BLOCKS_PER_TILE = SCHED_KEYS_PER_TILE // 64
+SCHED_OVERHEAD_TILES = 1  # cost of starting a sequence, in key tiles
+SCHED_MIN_CAP = 2  # smallest partition cost (tiles), so tiny problems are not shattered
 ROWS_PER_TILE = 128  # query rows (heads x draft tokens) handled by one worker
 
 
 def schedule_ref(cache_seqlens: np.ndarray, s_q: int, H: int, num_workers: int) -> Dict:
-    """Split-KV schedule: cut the concatenation of all sequences' blocks into
-    contiguous ranges of near-equal cost, one per partition.
+    """Split-KV schedule: cut the concatenation of all sequences' key tiles into
+    contiguous ranges of near-equal cost, one per partition.  Cuts fall on whole
+    tiles of SCHED_BLOCKS_PER_TILE blocks, so a split never leaves a ragged tile
+    except at a sequence's end.
 
-    Cost model: every block costs 1, and every sequence with at least one block
-    costs SCHED_OVERHEAD_BLOCKS extra, placed just before its first block.  Let
-    pre[b] be the total cost of sequences before b; block k of sequence b sits at
-    cost position pos = pre[b] + OVERHEAD + k.  With P = num_workers // T partitions
-    (T = ceil(s_q*H / 128) row tiles, each row tile scheduled identically) and
-    cap = max(SCHED_MIN_CAP, ceil(total_cost / P)), block (b, k) belongs to partition
-    floor(pos / cap).
+    Cost model: every key tile (up to 4 blocks) costs 1, and every sequence with at
+    least one block costs SCHED_OVERHEAD_TILES extra, placed just before its first
+    tile.  Let pre[b] be the total cost of sequences before b; tile j of sequence b
+    sits at cost position pos = pre[b] + OVERHEAD + j.  With P = num_workers // T
+    partitions (T = ceil(s_q*H / 128) row tiles, each row tile scheduled
+    identically) and cap = max(SCHED_MIN_CAP, ceil(total_cost / P)), tile (b, j)
+    and its blocks belong to partition floor(pos / cap).
 
     Returns a dict of int arrays:
       num_parts, num_tiles, cap, total_slots (scalars)
@@ -218,7 +222,8 @@ def schedule_ref(cache_seqlens: np.ndarray, s_q: int, H: int, num_workers: int) 
     T = -(-(s_q * H) // ROWS_PER_TILE)
     P = max(1, num_workers // T)
     nblk = np.where(seqlens > 0, -(-seqlens // BLOCK_SIZE), 0)
-    cost = np.where(nblk > 0, nblk + SCHED_OVERHEAD_BLOCKS, 0)
+    ntile = -(-nblk // SCHED_BLOCKS_PER_TILE)
+    cost = np.where(nblk > 0, ntile + SCHED_OVERHEAD_TILES, 0)
     pre = np.concatenate([[0], np.cumsum(cost)])  # [B+1]
     total = int(pre[-1])
     cap = max(SCHED_MIN_CAP, -(-total // P))
@@ -228,25 +233,25 @@ def schedule_ref(cache_seqlens: np.ndarray, s_q: int, H: int, num_workers: int) 
     for b in range(B):
         if nblk[b] == 0:
             continue
-        p0 = (pre[b] + SCHED_OVERHEAD_BLOCKS) // cap
-        p1 = (pre[b] + SCHED_OVERHEAD_BLOCKS + nblk[b] - 1) // cap
+        p0 = (pre[b] + SCHED_OVERHEAD_TILES) // cap
+        p1 = (pre[b] + SCHED_OVERHEAD_TILES + ntile[b] - 1) // cap
         first_part[b] = p0
         num_splits[b] = p1 - p0 + 1
     split_prefix = np.concatenate([[0], np.cumsum(num_splits)])[:B]
     total_slots = int(num_splits.sum())
 
-    # start of partition p: the first block whose position is >= p * cap
+    # start of partition p: the first tile whose position is >= p * cap
     part_start = np.tile(np.array([B, 0], dtype=np.int64), (P, 1))
     for p in range(P):
         target = p * cap
         for b in range(B):
             if nblk[b] == 0:
                 continue
-            first_pos = pre[b] + SCHED_OVERHEAD_BLOCKS
-            last_pos = first_pos + nblk[b] - 1
+            first_pos = pre[b] + SCHED_OVERHEAD_TILES
+            last_pos = first_pos + ntile[b] - 1
             if last_pos >= target:
-                k = max(0, target - first_pos)
-                part_start[p] = (b, k)
+                j = max(0, target - first_pos)
+                part_start[p] = (b, j * SCHED_BLOCKS_PER_TILE)
                 break
     part_end = np.empty_like(part_start)
     part_end[:-1] = part_start[1:]

@@ -98,7 +98,8 @@ def test_metadata_matches_oracle(name):
     B = w.B
     P = sc["num_parts"]
     assert meta[0] == 0x4D4C4131
-    assert list(meta[1:10]) == [B, w.s_q, w.H, P, sc["num_tiles"], sc["cap"], sc["total_slots"], workers, 4]
+    assert list(meta[1:10]) == [B, w.s_q, w.H, P, sc["num_tiles"], sc["cap"], sc["total_slots"], workers,
+                             O.SCHED_OVERHEAD_TILES]
     ps = meta[16 : 16 + 512].reshape(256, 2)[:P]
     pe = meta[16 + 512 : 16 + 1024].reshape(256, 2)[:P]
     assert np.array_equal(ps, sc["part_start"]) and np.array_equal(pe, sc["part_end"])

@@ -23,8 +23,12 @@ def check_valid(seqlens, s_q, H, workers):
         cost = 0
         for b, lo, hi, s in pieces:
             assert 0 <= lo < hi <= nblk[b]
+            # cuts fall on whole key tiles: a piece starts on a tile boundary and
+            # ends on one or at the sequence end
+            assert lo % O.SCHED_BLOCKS_PER_TILE == 0
+            assert hi % O.SCHED_BLOCKS_PER_TILE == 0 or hi == nblk[b]
             covered[b].append((s, lo, hi, p))
-            cost += hi - lo
+            cost += -(-(hi - lo) // O.SCHED_BLOCKS_PER_TILE)
         costs.append(cost)
     for b in range(B):
         parts = sorted(covered[b])
@@ -40,7 +44,7 @@ def check_valid(seqlens, s_q, H, workers):
     assert np.array_equal(sc["split_prefix"], np.concatenate([[0], np.cumsum(sc["num_splits"])[:-1]]))
     # each sequence is cut at most once per partition boundary
     assert sc["total_slots"] <= B + P - 1
-    # balance: no partition exceeds the cap (blocks only; the overhead sits before blocks)
+    # balance: no partition exceeds the cap (tiles only; the overhead sits before tiles)
     assert max(costs) <= sc["cap"]
     return sc
 
@@ -66,27 +70,27 @@ def test_workload_schedules_valid(name):
 
 
 def test_hand_worked_schedule():
-    """Two sequences of 5 and 3 blocks (n = 300, 129), 2 partitions, overhead 4:
-    costs 9 and 7, total 16, cap = max(8, 16/2) = 8.
-    Positions: seq0 blocks at 4..8, seq1 blocks at 13..15.
-    Block->partition: seq0 k=0..3 -> 0 (pos 4..7), k=4 -> 1 (pos 8); seq1 -> 1.
-    Partition 1 starts at position 8 = seq0 block 4."""
-    sc = O.schedule_ref(np.array([300, 129]), 1, 128, 2)
-    assert sc["cap"] == 8 and sc["num_parts"] == 2
-    assert sc["part_start"].tolist() == [[0, 0], [0, 4]]
-    assert sc["part_end"].tolist() == [[0, 4], [2, 0]]
+    """Two sequences of 16 and 3 blocks (n = 1000, 129), 2 partitions, tiles of 4
+    blocks, overhead 1 tile: 4 and 1 tiles, costs 5 and 2, total 7,
+    cap = max(2, ceil(7/2)) = 4.  Positions: seq0 tiles at 1..4, seq1's tile at 6.
+    Tile->partition: seq0 tiles 0..2 -> 0 (pos 1..3), tile 3 -> 1 (pos 4); seq1 -> 1.
+    Partition 1 starts at position 4 = seq0 tile 3 = block 12."""
+    sc = O.schedule_ref(np.array([1000, 129]), 1, 128, 2)
+    assert sc["cap"] == 4 and sc["num_parts"] == 2
+    assert sc["part_start"].tolist() == [[0, 0], [0, 12]]
+    assert sc["part_end"].tolist() == [[0, 12], [2, 0]]
     assert sc["num_splits"].tolist() == [2, 1]
     assert sc["first_part"].tolist() == [0, 1]
     assert sc["split_prefix"].tolist() == [0, 2]
-    assert O.pieces_of_partition(sc, 0) == [(0, 0, 4, 0)]
-    assert O.pieces_of_partition(sc, 1) == [(0, 4, 5, 1), (1, 0, 3, 0)]
+    assert O.pieces_of_partition(sc, 0) == [(0, 0, 12, 0)]
+    assert O.pieces_of_partition(sc, 1) == [(0, 12, 16, 1), (1, 0, 3, 0)]
 
 
 def test_min_cap_keeps_tiny_problems_whole():
     sc = O.schedule_ref(np.array([37, 130]), 1, 16, 74)
-    # cost 1+4 and 3+4 = 12 -> cap 8: partition 0 holds seq0 and seq1's first
-    # block... positions: seq0 block at 4, seq1 blocks at 9,10,11 -> partitions 0,1,1,1
-    assert sc["cap"] == 8
+    # 1 and 3 blocks = 1 tile each, costs 2 and 2, total 4 -> cap = max(2, 1) = 2:
+    # seq0's tile at position 1 -> partition 0, seq1's tile at 3 -> partition 1
+    assert sc["cap"] == 2
     assert sc["num_splits"].tolist() == [1, 1]
     assert sc["first_part"].tolist() == [0, 1]
 
