@@ -420,17 +420,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         }
       };
       // Ring order per piece: QK(0), then QK(t) followed by PV(t - 1), then PV(last).
-      while (ok && walk.next(cur)) {
+      // The next piece is looked up one piece ahead and its first 32 block ids are
+      // loaded during the current piece's last tile, so a piece starts without
+      // waiting on the block table.
+      Piece nxt{};
+      bool have = walk.next(cur);
+      bool have_nxt = have && walk.next(nxt);
+      if (have) {
         bt = p.block_table + (int64_t)cur.b * p.max_blocks;
-        id_chunks = 0;
         id_pending = fetch_id(lane);
+      }
+      while (ok && have) {
+        id_chunks = 0;
         const int nt = num_tiles(cur);
+        int id_next = 0;
         for (int t = 0; t < nt && ok; ++t) {
+          if (t == nt - 1 && have_nxt) {
+            const int32_t* btn = p.block_table + (int64_t)nxt.b * p.max_blocks;
+            id_next = (lane < nxt.k_hi - nxt.k_lo) ? clamp_block_id(p, btn[nxt.k_lo + lane]) : 0;
+          }
           issue_qk(t);
           if (t >= 1 && ok) issue_pv(cur, cur_base, t - 1);
         }
         if (ok) issue_pv(cur, cur_base, nt - 1);
         cur_base = (cur_base + 32 * id_chunks) % kIdRing;
+        have = have_nxt;
+        if (have) {
+          cur = nxt;
+          bt = p.block_table + (int64_t)cur.b * p.max_blocks;
+          id_pending = id_next;
+          have_nxt = walk.next(nxt);
+        }
       }
     }
     // =======================================================================
