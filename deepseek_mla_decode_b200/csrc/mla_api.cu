@@ -18,6 +18,7 @@ cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, int max_
 cudaError_t decode_kernel_setup(int device);
 cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
                           const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
+                          const CUtensorMap& tm_out, const CUtensorMap& tm_part,
                           const int32_t* block_table, int max_blocks, const int32_t* seqlens,
                           const int32_t* meta, int64_t num_blocks, int B, int s_q, int H, float scale,
                           int causal, void* out, float* lse, float* part_o, float* part_lse,
@@ -95,9 +96,9 @@ int parts_for(int num_workers, int s_q, int H) {
 }
 
 bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
-            const cuuint32_t* box) {
+            const cuuint32_t* box, CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   cuuint32_t es[4] = {1, 1, 1, 1};
-  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
+  return g_encode(m, dt, rank, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -236,7 +237,22 @@ mla_status_t launch_attention(const void* q_nope, const void* q_pe, const void* 
   }
   float* part_o = static_cast<float*>(workspace);
   float* part_lse = part_o + g.slots * g.M * mla::kDLatent;
-  if (mla::launch_decode(tm_kv, tm_kv2, tm_qn, tm_qp, block_table, max_blocks, cache_seqlens,
+  // Output views for the epilogue's TMA stores: rows past M of a sequence are clipped.
+  CUtensorMap tm_out, tm_part;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)mla::kDLatent, (cuuint64_t)g.M, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)mla::kDLatent * 2, (cuuint64_t)g.M * mla::kDLatent * 2};
+    cuuint32_t box[3] = {64, 64, 1};
+    if (!encode(&tm_out, out, 3, dims, strides, box)) return MLA_ERR_INVALID_ARG;
+  }
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)mla::kDLatent, (cuuint64_t)g.M, (cuuint64_t)g.slots};
+    cuuint64_t strides[2] = {(cuuint64_t)mla::kDLatent * 4, (cuuint64_t)g.M * mla::kDLatent * 4};
+    cuuint32_t box[3] = {32, 64, 1};
+    if (!encode(&tm_part, part_o, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
+      return MLA_ERR_INVALID_ARG;
+  }
+  if (mla::launch_decode(tm_kv, tm_kv2, tm_qn, tm_qp, tm_out, tm_part, block_table, max_blocks, cache_seqlens,
                          static_cast<const int32_t*>(metadata), num_blocks, B, s_q, H, softmax_scale, causal != 0,
                          out, lse, part_o, part_lse, status, 2 * g.P * g.T, s) != cudaSuccess)
     return MLA_ERR_CUDA;

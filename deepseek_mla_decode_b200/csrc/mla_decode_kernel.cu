@@ -66,6 +66,8 @@ struct Params {
   CUtensorMap tm_kv2;  // same memory as [num_blocks][9][64][64], box {64, 64, 2, 1}, SW128
   CUtensorMap tm_qn;  // [B*M][512] bf16, box {64, 64}, SW128
   CUtensorMap tm_qp;  // [B*M][64] bf16, box {64, 64}, SW128
+  CUtensorMap tm_out;   // out as [B][M][512] bf16, box {64, 64, 1}, SW128 (TMA store)
+  CUtensorMap tm_part;  // partial outputs as [slots][M][512] fp32, box {32, 64, 1}, SW128
   const int32_t* block_table;
   const int32_t* seqlens;
   const int32_t* meta;
@@ -237,6 +239,15 @@ __device__ __forceinline__ void tma_load_4d_cg2_if(bool on, uint32_t dst, const 
       "r"((uint32_t)on)
       : "memory");
 }
+__device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
@@ -314,6 +325,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     prefetch_tmap(&p.tm_kv2);
     prefetch_tmap(&p.tm_qn);
     prefetch_tmap(&p.tm_qp);
+    prefetch_tmap(&p.tm_out);
+    prefetch_tmap(&p.tm_part);
   }
   tc_fence_before();
   __syncthreads();
@@ -750,7 +763,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
         const float lse_val =
             bad ? nanf_ : ((l32_row > 0.f) ? (m_used + __log2f(l32_row)) * 0.69314718055994531f : -INFINITY);
-        const int dim0 = 256 * g + 128 * hk;
         const int64_t orow = (int64_t)pc.b * p.M + grow;
         const int64_t slot = (int64_t)split_base + pc.split;
         ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1, false);
@@ -760,30 +772,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         const uint32_t to = tmem + kTmemO + 128 * g + lane_off;
         // a bad piece's rows become NaN: scaling by NaN turns every value into NaN
         const float sc = bad ? nanf_ : inv_l;
-        auto emit = [&](const uint32_t (&o)[32], int c) {
-          if (!row_valid) return;
-          auto v = [&](int j) { return __uint_as_float(o[j]) * sc; };
-          if (direct) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDLatent + dim0 + c);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(pack_bf16x2(v(8 * j), v(8 * j + 1)), pack_bf16x2(v(8 * j + 2), v(8 * j + 3)),
-                                  pack_bf16x2(v(8 * j + 4), v(8 * j + 5)), pack_bf16x2(v(8 * j + 6), v(8 * j + 7)));
-          } else {
-            float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * p.M + grow) * kDLatent + dim0 + c);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) dst[j] = make_float4(v(4 * j), v(4 * j + 1), v(4 * j + 2), v(4 * j + 3));
-          }
-        };
-        // two 32-column TMEM loads in flight per wait
+        // The output leaves through TMA stores staged in the P buffer (unused until the
+        // next piece's first P): per round every thread writes 128 bytes of its row
+        // (64 bf16 or 32 fp32 columns) into box 2g + hk, laid out [64 rows][128 B] with
+        // the 128-byte swizzle, and one thread stores the four boxes.  Rows past M are
+        // clipped by the tensor map.
+        const uint32_t srow = sP + (2 * g + hk) * kChunkBytes + m * 128;
+        const int rounds = direct ? 2 : 4;
+        const int y0 = tile_row0 + kRowsPerCta * (int)rank;
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 64) {
-          uint32_t o0[32], o1[32];
-          tmem_ld32(to + c, o0);
-          tmem_ld32(to + c + 32, o1);
-          tmem_wait_ld();
-          emit(o0, c);
-          emit(o1, c + 32);
+        for (int r = 0; r < rounds; ++r) {
+          uint32_t w[32];
+          if (direct) {
+            uint32_t o0[32], o1[32];
+            tmem_ld32(to + 64 * r, o0);
+            tmem_ld32(to + 64 * r + 32, o1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              w[k] = pack_bf16x2(__uint_as_float(o0[2 * k]) * sc, __uint_as_float(o0[2 * k + 1]) * sc);
+              w[16 + k] = pack_bf16x2(__uint_as_float(o1[2 * k]) * sc, __uint_as_float(o1[2 * k + 1]) * sc);
+            }
+          } else {
+            tmem_ld32(to + 32 * r, w);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * sc);
+          }
+          if (r > 0) named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);  // previous round's boxes were read
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(srow + ((q ^ (m & 7)) << 4)),
+                         "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
+                         : "memory");
+          fence_proxy_async_smem();
+          named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
+          if (st == 0 && y0 < p.M) {  // a CTA whose 64 rows all lie past M stores nothing
+#pragma unroll
+            for (int bx = 0; bx < 4; ++bx) {
+              const int gg = bx >> 1, hh = bx & 1;
+              if (direct)
+                tma_store_3d(&p.tm_out, sP + bx * kChunkBytes, 256 * gg + 128 * hh + 64 * r, y0, pc.b);
+              else
+                tma_store_3d(&p.tm_part, sP + bx * kChunkBytes, 256 * gg + 128 * hh + 32 * r, y0, (int)slot);
+            }
+            bulk_commit();
+            bulk_wait_read_all();
+          }
         }
         if (row_valid && hk == 0 && g == 0) {
           if (direct)
@@ -804,6 +839,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
   }
 
   // ---- teardown ------------------------------------------------------------
+  if (warp == kSoftmaxWarp0 && lane == 0) bulk_wait_all();  // the epilogue's TMA stores landed
   tc_fence_before();
   __syncthreads();
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -826,6 +862,7 @@ cudaError_t decode_kernel_setup(int device) {
 
 cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
                           const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
+                          const CUtensorMap& tm_out, const CUtensorMap& tm_part,
                           const int32_t* block_table, int max_blocks, const int32_t* seqlens,
                           const int32_t* meta, int64_t num_blocks, int B, int s_q, int H, float scale,
                           int causal, void* out, float* lse, float* part_o, float* part_lse,
@@ -835,6 +872,8 @@ cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
   prm.tm_kv2 = tm_kv2;
   prm.tm_qn = tm_qn;
   prm.tm_qp = tm_qp;
+  prm.tm_out = tm_out;
+  prm.tm_part = tm_part;
   prm.block_table = block_table;
   prm.seqlens = seqlens;
   prm.meta = meta;
