@@ -12,9 +12,9 @@
 namespace mla {
 cudaError_t launch_metadata(const int32_t* seqlens, int B, int s_q, int H, int num_workers, int32_t* meta,
                             cudaStream_t stream);
-cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, int max_blocks, int B, int M,
+cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, int max_blocks, int B, int M, int P,
                            const float* part_o, const float* part_lse, void* out, float* lse,
-                           int32_t* status, cudaStream_t stream);
+                           cudaStream_t stream);
 cudaError_t decode_kernel_setup(int device);
 cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
                           const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
@@ -300,8 +300,10 @@ mla_status_t mla_decode_combine(const int32_t* cache_seqlens, int max_blocks, in
   const int64_t slots = mla::ws_slots(B, num_workers_for(sms));
   const float* part_o = static_cast<const float*>(workspace);
   const float* part_lse = part_o + slots * M * mla::kDLatent;
-  if (mla::launch_combine(static_cast<const int32_t*>(metadata), cache_seqlens, max_blocks, B, M, part_o, part_lse,
-                          out, lse, status, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  (void)status;  // the combine raises no error of its own
+  if (mla::launch_combine(static_cast<const int32_t*>(metadata), cache_seqlens, max_blocks, B, M,
+                          parts_for(num_workers_for(sms), s_q, H), part_o, part_lse, out, lse,
+                          static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;
 }
@@ -322,8 +324,8 @@ mla_status_t mla_decode(const void* q_nope, const void* q_pe, const void* kv_cac
   if (st != MLA_OK) return st;
   const float* part_o = static_cast<const float*>(workspace);
   const float* part_lse = part_o + g.slots * g.M * mla::kDLatent;
-  if (mla::launch_combine(static_cast<const int32_t*>(metadata), cache_seqlens, max_blocks, B, g.M, part_o,
-                          part_lse, out, lse, status, s) != cudaSuccess)
+  if (mla::launch_combine(static_cast<const int32_t*>(metadata), cache_seqlens, max_blocks, B, g.M, g.P, part_o,
+                          part_lse, out, lse, s) != cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;
 }

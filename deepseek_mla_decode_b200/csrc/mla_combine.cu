@@ -7,9 +7,11 @@
 // the softmax_lse side output).  HBM-bound: one warp per query row streams the S
 // partial rows with 16-byte loads and writes the bf16 row once.
 //
-// The kernel also finishes rows the decode kernel does not own: sequences with no
-// visible key (out = 0, lse = -inf) and sequences with an invalid length (NaN and an
-// error bit in the status word).
+// Grid (P, ceil(M / 8)): block x = p looks at partition p's first block; a split
+// sequence is exactly one whose cut opens a partition mid-sequence, and the first such
+// partition (first_part + 1) owns its merge, so only blocks with work touch memory.
+// Rows of sequences that no partition covers (no visible key, invalid length) are
+// written by the attention kernel.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -29,28 +31,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
     const int32_t* __restrict__ meta, const int32_t* __restrict__ seqlens, int max_blocks,
     int B, int M, const float* __restrict__ part_o, const float* __restrict__ part_lse,
-    __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int32_t* status) {
-  const int b = blockIdx.x;
+    __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  const int part = blockIdx.x;
+  if (part == 0) return;
+  const int b = meta[off_part_start() + 2 * part];
+  if (b >= B || meta[off_part_start() + 2 * part + 1] == 0) return;  // partition opens a sequence
+  if (meta[off_first_part(B) + b] + 1 != part) return;              // a later cut of the same sequence
+  const int n = seqlens[b];
+  if (n < 0 || (int64_t)n > (int64_t)max_blocks * kBlockSize) return;  // rows written as NaN already
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.y * kWarps + warp;
   if (row >= M) return;
-  const int n = seqlens[b];
   const int ns = meta[off_num_splits(B) + b];
   uint2* orow = reinterpret_cast<uint2*>(out + ((int64_t)b * M + row) * kDLatent);
-  const bool bad_len = n < 0 || (int64_t)n > (int64_t)max_blocks * kBlockSize;
-  if (bad_len || ns == 0) {
-    const float v = bad_len ? __int_as_float(0x7fc00000) : 0.0f;
-    const uint32_t pv = pack_bf16x2(v, v);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) orow[k * 32 + lane] = make_uint2(pv, pv);
-    if (lane == 0) {
-      lse[(int64_t)b * M + row] = bad_len ? __int_as_float(0x7fc00000) : -INFINITY;
-      if (bad_len && row == 0 && status) atomicOr(status, kErrSeqlen);
-    }
-    return;
-  }
-  if (ns == 1) return;  // written by the decode kernel
-
   const int64_t slot0 = meta[off_split_prefix(B) + b];
   // pass 1: max and sum over the partial lse values (every lane redundantly)
   float m = -INFINITY;
@@ -96,11 +89,11 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
 }  // namespace
 
 cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, int max_blocks, int B,
-                           int M, const float* part_o, const float* part_lse, void* out, float* lse,
-                           int32_t* status, cudaStream_t stream) {
-  dim3 grid(B, (M + kWarps - 1) / kWarps);
+                           int M, int P, const float* part_o, const float* part_lse, void* out, float* lse,
+                           cudaStream_t stream) {
+  dim3 grid(P, (M + kWarps - 1) / kWarps);
   combine_kernel<<<grid, kWarps * 32, 0, stream>>>(meta, seqlens, max_blocks, B, M, part_o, part_lse,
-                                                   reinterpret_cast<__nv_bfloat16*>(out), lse, status);
+                                                   reinterpret_cast<__nv_bfloat16*>(out), lse);
   return cudaGetLastError();
 }
 

@@ -271,6 +271,28 @@ __device__ __forceinline__ int clamp_block_id(const Params& p, int32_t id) {
   return id;
 }
 
+// Rows of sequences that no partition covers: no visible key (out 0, lse -inf) or an
+// invalid length (NaN and the status bit).  Partition `part` takes the sequences b with
+// b % P == part; the 32 lanes of one warp write this CTA's 64 rows [y0, y0 + 64).
+__device__ __forceinline__ void write_orphan_rows(const Params& p, int part, int P, int y0, int lane) {
+  for (int b = part; b < p.B; b += P) {
+    const int n = p.seqlens[b];
+    const bool bad_len = n < 0 || (int64_t)n > (int64_t)p.max_blocks * kBlockSize;
+    if (!bad_len && n > 0) continue;
+    const float v = bad_len ? __int_as_float(0x7fc00000) : 0.0f;
+    const uint32_t pv = pack_bf16x2(v, v);
+    for (int i = lane; i < kRowsPerCta * (kDLatent / 8); i += 32) {  // 16-byte units
+      const int row = y0 + i / (kDLatent / 8);
+      if (row < p.M)
+        reinterpret_cast<uint4*>(p.out + ((int64_t)b * p.M + row) * kDLatent)[i % (kDLatent / 8)] =
+            make_uint4(pv, pv, pv, pv);
+    }
+    for (int r = lane; r < kRowsPerCta; r += 32)
+      if (y0 + r < p.M) p.lse[(int64_t)b * p.M + y0 + r] = bad_len ? __int_as_float(0x7fc00000) : -INFINITY;
+    if (bad_len && lane == 0) set_status(p, kErrSeqlen);
+  }
+}
+
 // ===========================================================================
 // the kernel
 // ===========================================================================
@@ -465,6 +487,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           have_nxt = walk.next(nxt);
         }
       }
+      // With its loads issued, producer warp 0 writes the rows that no partition
+      // covers while the last tiles are still being computed.
+      if (pi == 0) write_orphan_rows(p, part, P, tile_row0 + kRowsPerCta * (int)rank, lane);
     }
     // =======================================================================
     // Q loader (both CTAs): Q of piece k + 1 is loaded as soon as the last QK of

@@ -138,11 +138,13 @@ mla_status_t mla_decode(const void* q_nope, const void* q_pe, const void* kv_cac
  *
  * mla_decode_attention: the split-KV attention kernel.  Sequences processed in one
  *   piece get their out / lse rows written directly; pieces of split sequences write
- *   normalised fp32 partial outputs and their lse into the workspace.
+ *   normalised fp32 partial outputs and their lse into the workspace.  It also writes
+ *   the rows of sequences with no visible key (0 / -inf) and of sequences with an
+ *   invalid length (NaN, MLA_DEVICE_ERR_SEQLEN).
  * mla_decode_combine: the LSE-combine kernel (split-K merge, "DeepSeek speed test /
  *   FA3" article section 2.1): for every split sequence, lse = ln sum_s exp(lse_s) and
- *   out = sum_s exp(lse_s - lse) O_s; it also writes the rows of sequences with no
- *   visible key (0 / -inf) and of sequences with an invalid length (NaN).
+ *   out = sum_s exp(lse_s - lse) O_s.  Only split sequences are touched; `status` is
+ *   accepted for symmetry and never written.
  */
 mla_status_t mla_decode_attention(const void* q_nope, const void* q_pe, const void* kv_cache,
                                   int64_t num_blocks, const int32_t* block_table, int max_blocks,
