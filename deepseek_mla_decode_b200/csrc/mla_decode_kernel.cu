@@ -187,14 +187,6 @@ __device__ __forceinline__ bool wait_bar(Ctrl* c, const Params& p, uint32_t bar,
   }
 }
 
-__device__ __forceinline__ void tma_load_2d_cg2(uint32_t dst, const void* tmap, uint32_t bar_cluster,
-                                                int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1)
-      : "memory");
-}
 // Predicated forms: the whole warp executes the instruction and only lanes with
 // `on` set issue it, so the issuing warp never diverges around the issue.
 __device__ __forceinline__ void umma_2sm_if(bool on, uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
@@ -227,6 +219,15 @@ __device__ __forceinline__ void tma_load_3d_cg2_if(bool on, uint32_t dst, const 
       "@q cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];\n\t}" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"((uint32_t)on)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_cg2_if(bool on, uint32_t dst, const void* tmap, uint32_t bar_cluster,
+                                                   int c0, int c1) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+      "@q cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];\n\t}" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"((uint32_t)on)
       : "memory");
 }
 __device__ __forceinline__ void tma_load_4d_cg2_if(bool on, uint32_t dst, const void* tmap, uint32_t bar_cluster,
@@ -496,23 +497,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     // piece k has completed, while the MMAs still work through the PV of piece k.
     // =======================================================================
     else if (warp == kQWarp) {
-      if (lane == 0) {
-        PieceWalker walk(p, part);
-        Piece pc;
-        int npieces = 0;
-        const uint32_t q_full_l = mapa_shared(smem_u32(&ctrl.q_full), 0);
-        while (walk.next(pc)) {
-          if (npieces > 0 && !wait_bar(&ctrl, p, smem_u32(&ctrl.q_empty), (npieces - 1) & 1, false)) break;
-          const int row_base = pc.b * p.M + tile_row0 + kRowsPerCta * (int)rank;
-          if (leader) mbar_arrive_expect_tx(smem_u32(&ctrl.q_full), 2 * kQBytes);
-          for (int c = 0; c < kQChunks; ++c) {
-            if (c < 8)
-              tma_load_2d_cg2(sQ + c * kChunkBytes, &p.tm_qn, q_full_l, 64 * c, row_base);
-            else
-              tma_load_2d_cg2(sQ + c * kChunkBytes, &p.tm_qp, q_full_l, 0, row_base);
-          }
-          ++npieces;
-        }
+      // the whole warp waits (converged); lanes 0..8 each issue one 64-column box
+      PieceWalker walk(p, part);
+      Piece pc;
+      int npieces = 0;
+      const uint32_t q_full_l = mapa_shared(smem_u32(&ctrl.q_full), 0);
+      while (walk.next(pc)) {
+        if (npieces > 0 &&
+            !__shfl_sync(0xffffffffu, wait_bar(&ctrl, p, smem_u32(&ctrl.q_empty), (npieces - 1) & 1, false), 0))
+          break;
+        const int row_base = pc.b * p.M + tile_row0 + kRowsPerCta * (int)rank;
+        expect_tx_if(lane == 0 && leader, smem_u32(&ctrl.q_full), 2 * kQBytes);
+        __syncwarp();
+        const int c = lane < kQChunks ? lane : 0;
+        tma_load_2d_cg2_if(lane < kQChunks, sQ + c * kChunkBytes, c < 8 ? (const void*)&p.tm_qn : (const void*)&p.tm_qp,
+                           q_full_l, c < 8 ? 64 * c : 0, row_base);
+        ++npieces;
       }
     }
     // =======================================================================
