@@ -19,10 +19,10 @@
 //       all 256 dims of that half.
 // O uses TMEM columns [0, 256), the two S buffers [256, 384) and [384, 512).
 //
-// Warp roles (416 threads): warps 0, 2, 3 = TMA producers (alternate ring stages),
-// warp 1 = MMA issuer (leader CTA only) and TMEM owner, warps 4..11 = softmax /
-// correction / epilogue (thread = one row x 64 keys of S, one row x 128 dims of O),
-// warp 12 = Q loader.
+// Warp roles (448 threads): warps 0, 2, 3, 13 = TMA producers (stage k is issued by
+// producer k % 4), warp 1 = MMA issuer (leader CTA only) and TMEM owner, warps 4..11 =
+// softmax / correction / epilogue (thread = one row x 64 keys of S, one row x 128 dims
+// of O), warp 12 = Q loader.
 // Every mbarrier wait is bounded; a
 // timeout sets MLA_DEVICE_ERR_TIMEOUT, raises a CTA-wide abort flag and the kernel
 // drains and returns.
@@ -39,8 +39,8 @@ using namespace ptx;
 
 namespace {
 
-constexpr int kNumThreads = 416;
-constexpr int kNumProducers = 3;  // warps 0, 2, 3
+constexpr int kNumThreads = 448;
+constexpr int kNumProducers = 4;  // warps 0, 2, 3, 13
 constexpr int kMmaWarp = 1;
 constexpr int kSoftmaxWarp0 = 4;   // warps 4..11
 constexpr int kQWarp = 12;
@@ -99,7 +99,7 @@ struct __align__(8) Ctrl {
   float red_sum[4][64];   // sum of the bf16-rounded weights (normalises the output)
   float red_sum32[4][64]; // sum of the fp32 weights (gives the lse)
   int bad_piece;
-  int block_ids[3][128];  // each producer's window of physical block ids (current and previous piece)
+  int block_ids[4][128];  // each producer's window of the current piece's physical block ids
 };
 constexpr int kIdRing = 128;
 
@@ -359,12 +359,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
 
   if (tile < T) {
     // =======================================================================
-    // producers: warps 0, 2 and 3 own ring stages k % 3 == 0, 1, 2 (one issuing
-    // warp sustains only ~half the L2 -> SM bandwidth a CTA needs; several warps
-    // issuing alternate stages of the same ring lift that limit).  Warp 0 also loads Q.
+    // producers: warps 0, 2, 3 and 13 own ring stages k % 4 == 0, 1, 2, 3 (one
+    // issuing warp sustains only ~half the L2 -> SM bandwidth a CTA needs; several
+    // warps issuing alternate stages of the same ring lift that limit).
     // =======================================================================
-    if (warp == 0 || warp == 2 || warp == 3) {
-      const int pi = (warp == 0) ? 0 : warp - 1;
+    if (warp == 0 || warp == 2 || warp == 3 || warp == 13) {
+      const int pi = (warp == 0) ? 0 : (warp == 13 ? 3 : warp - 1);
       int32_t* idwin = ctrl.block_ids[pi];
       PieceWalker walk(p, part);
       uint32_t it = 0;

@@ -66,6 +66,74 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
   int32_t* num_splits = meta + off_num_splits(B);
   int32_t* split_prefix = meta + off_split_prefix(B);
 
+  // ---- fast path: the whole batch fits one pass of the block ------------------
+  // (same arithmetic as the general passes below, with one load of the lengths and
+  // one scan of the costs instead of two)
+  if (B <= kThreads) {
+    const int b = tid;
+    const int n = (b < B) ? seqlens[b] : 0;
+    const int nb = n > 0 ? (n + kBlockSize - 1) / kBlockSize : 0;
+    const int64_t nt = (nb + kBlocksPerTile - 1) / kBlocksPerTile;
+    const int64_t cost = nb > 0 ? nt + kSchedOverheadTiles : 0;
+    int64_t total;
+    const int64_t pre = block_exclusive_scan(cost, scratch, &total);
+    int64_t cap = (total + P - 1) / P;
+    if (cap < kSchedMinCap) cap = kSchedMinCap;
+    for (int q = tid; q < kMaxWorkers; q += kThreads) {
+      part_start[2 * q] = B;
+      part_start[2 * q + 1] = 0;
+    }
+    __syncthreads();
+    int64_t ns = 0;
+    if (b < B) {
+      nblk_out[b] = nb;
+      if (nb > 0) {
+        const int64_t first_pos = pre + kSchedOverheadTiles;
+        const int64_t p0 = first_pos / cap;
+        const int64_t p1 = (first_pos + nt - 1) / cap;
+        first_part[b] = (int32_t)p0;
+        ns = p1 - p0 + 1;
+        const int64_t lo = (pre + cap - 1) / cap;
+        const int64_t hi = (pre + cost - 1) / cap;
+        for (int64_t q = lo; q <= hi && q < P; ++q) {
+          const int64_t j = q * cap - first_pos;  // first tile of partition q
+          part_start[2 * q] = b;
+          part_start[2 * q + 1] = (int32_t)(j > 0 ? j * kBlocksPerTile : 0);
+        }
+      } else {
+        first_part[b] = 0;
+      }
+      num_splits[b] = (int32_t)ns;
+    }
+    int64_t total_slots;
+    const int64_t ex = block_exclusive_scan(ns, scratch, &total_slots);
+    if (b < B) split_prefix[b] = (int32_t)ex;
+    __syncthreads();
+    for (int q = tid; q < kMaxWorkers; q += kThreads) {
+      if (q + 1 < P) {
+        part_end[2 * q] = part_start[2 * (q + 1)];
+        part_end[2 * q + 1] = part_start[2 * (q + 1) + 1];
+      } else {
+        part_end[2 * q] = B;
+        part_end[2 * q + 1] = 0;
+      }
+    }
+    if (tid == 0) {
+      meta[kHdrMagic] = kMetaMagic;
+      meta[kHdrB] = B;
+      meta[kHdrSq] = s_q;
+      meta[kHdrH] = H;
+      meta[kHdrNumParts] = P;
+      meta[kHdrNumTiles] = T;
+      meta[kHdrCap] = (int32_t)cap;
+      meta[kHdrTotalSlots] = (int32_t)total_slots;
+      meta[kHdrNumWorkers] = num_workers;
+      meta[kHdrOverhead] = kSchedOverheadTiles;
+      for (int i = kHdrOverhead + 1; i < kHdrWords; ++i) meta[i] = 0;
+    }
+    return;
+  }
+
   // ---- pass 1: total cost -------------------------------------------------
   int64_t total = 0;
   for (int base = 0; base < B; base += kThreads) {

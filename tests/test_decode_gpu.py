@@ -87,6 +87,26 @@ def test_deterministic():
 # ---------------------------------------------------------------------------
 # schedule: bit-exact against the oracle
 # ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B", [1023, 1024, 1025, 3000])
+def test_metadata_matches_oracle_large_batch(B):
+    """Batches around and beyond one pass of the scheduler block (1024 sequences):
+    the single-pass and multi-pass paths give the oracle's schedule word for word."""
+    rng = np.random.default_rng(B)
+    seqlens = rng.integers(0, 3000, size=B).astype(np.int64)
+    seqlens[rng.random(B) < 0.05] = 0
+    t = torch.from_numpy(seqlens.astype(np.int32)).cuda()
+    meta = mla.get_metadata(t, 1, 128).cpu().numpy()
+    workers = min(mla.device_sm_count() // 2, 256)
+    sc = O.schedule_ref(seqlens, 1, 128, workers)
+    P = sc["num_parts"]
+    assert list(meta[1:9]) == [B, 1, 128, P, sc["num_tiles"], sc["cap"], sc["total_slots"], workers]
+    assert np.array_equal(meta[16 : 16 + 512].reshape(256, 2)[:P], sc["part_start"])
+    assert np.array_equal(meta[16 + 512 : 16 + 1024].reshape(256, 2)[:P], sc["part_end"])
+    base = 16 + 1024
+    for i, key in enumerate(["nblk", "first_part", "num_splits", "split_prefix"]):
+        assert np.array_equal(meta[base + i * B : base + (i + 1) * B], sc[key]), key
+
+
 @pytest.mark.parametrize("name", ["tiny", "decode_b64", "mtp_b128_sq2", "serving_b256", "long_b4"])
 def test_metadata_matches_oracle(name):
     w = WORKLOADS[name]
