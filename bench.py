@@ -60,6 +60,23 @@ def algorithmic_work(seqlens, s_q, H, causal):
     return flops, cache_bytes, cache_bytes + q_bytes + out_bytes
 
 
+def max_over_ranks(values, world, device, dist=None):
+    """Element-wise max of `values` over all ranks of the process group (the identity
+    on one rank).  Every rank must call it with the same number of values."""
+    import torch
+
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def whole_job_rate(world, work_per_rank, ms):
+    """Throughput of the whole job: every rank did `work_per_rank` in at most `ms`
+    (the slowest rank's time), so the job did world * work in that time."""
+    return world * work_per_rank / (ms * 1e-3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -308,10 +325,7 @@ def main():
     att_ms = sum(ev_a[k][0].elapsed_time(ev_a[k][1]) for k in range(K))
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} in the timed region")
-    t = torch.tensor([step_ms, att_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms, att_ms = float(t[0]), float(t[1])
+    step_ms, att_ms = max_over_ranks([step_ms, att_ms], world, dev, dist)
 
     # ---- end to end through the public API with host buffers ---------------
     e2e = None
@@ -347,11 +361,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te[0])
-        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+        (e2e_ms,) = max_over_ranks([e2e_ms], world, dev, dist)
+        e2e = {"value": whole_job_rate(world, flops, e2e_ms) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
 
     if rank != 0:
@@ -362,7 +373,7 @@ def main():
     hbm_peak, tc_peak, tc_sustained, peak_src = load_peaks()
     ms = step_ms / K
     att_avg_s = att_ms / K * 1e-3
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = whole_job_rate(world, flops, ms) / 1e12
     t_hbm = cache_bytes / (hbm_peak * 1e9)
     t_tc = flops / (tc_peak * 1e12)
     bound = "hbm" if t_hbm >= t_tc else "tensor"
