@@ -108,7 +108,7 @@ struct Piece {
 };
 
 // Walks the pieces of one partition.  Pieces of sequences whose length is invalid
-// are skipped consistently by every role (the combine kernel writes their NaN rows).
+// are skipped consistently by every role (producer warp 0 writes their NaN rows).
 struct PieceWalker {
   const Params* p;
   int cb, ck, be, ke;
