@@ -6,8 +6,10 @@
                     [--impl ours|reference]
 
 Prints one JSON line (rank 0).  Device times come from CUDA events on the launching
-stream, summed over exactly K timed steps; an L2 flush (a 256 MB write, twice the L2)
-runs before every step outside the timed events.  Multi-GPU runs (torchrun) are
+stream, summed over exactly K timed steps; an L2 flush (a 256 MB write, then a 256 MB
+read that evicts the dirty lines) runs before every step outside the timed events.  The
+line also carries the attention kernel's roofline figures for the other decode
+configurations (per_workload).  Multi-GPU runs (torchrun) are
 independent replicas of the same workload per GPU (weak scaling; the path has no
 exchange step): value = all ranks' FLOPs / max-over-ranks time.
 
@@ -58,6 +60,11 @@ def algorithmic_work(seqlens, s_q, H, causal):
     q_bytes = B * s_q * H * D_QK * 2
     out_bytes = B * s_q * H * D_LATENT * 2 + B * s_q * H * 4
     return flops, cache_bytes, cache_bytes + q_bytes + out_bytes
+
+
+def metric_name(w):
+    """The metric string both arms print, so their lines can be divided."""
+    return f"MLA decode TFLOP/s ({w.name}: B={w.B}, s_q={w.s_q}, H={w.H})"
 
 
 def max_over_ranks(values, world, device, dist=None):
@@ -145,7 +152,7 @@ class ClockSampler:
                 self.reasons |= fn(self.h)
             except Exception:
                 pass
-            time.sleep(0.01)
+            time.sleep(0.002)
 
     def __enter__(self):
         if self.nv is not None:
@@ -206,6 +213,165 @@ def cpu_cores():
 
 
 # ---------------------------------------------------------------------------
+# device timing
+# ---------------------------------------------------------------------------
+class L2Flush:
+    """Before every step, outside the timed events: a 256 MB write (twice the L2) and
+    then a 256 MB read of another buffer.  The read evicts the dirty lines the write
+    left, so their write-back does not land inside the next timed kernel, and the step
+    starts with none of its own inputs in L2."""
+
+    DESCRIPTION = ("256 MB write then 256 MB read before every step, outside the timed events "
+                   "(inputs come from HBM; no dirty lines are written back inside the timed kernel)")
+
+    def __init__(self, dev):
+        import torch
+
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        import torch
+
+        self.w.zero_()
+        torch.sum(self.r, out=self.sink)
+
+
+class DeviceRun:
+    """One workload resident on the device, stepped through the C ABI: schedule,
+    attention and LSE combine, each bracketed by CUDA events on the launching stream."""
+
+    def __init__(self, mla, inp, dev):
+        import torch
+
+        self.mla, self.inp, self.dev = mla, inp, dev
+
+        def bf16(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+        self.q_nope, self.q_pe, self.kv = bf16(inp.q_nope), bf16(inp.q_pe), bf16(inp.kv_cache)
+        self.table = torch.from_numpy(inp.block_table).to(dev)
+        self.seqlens = torch.from_numpy(inp.cache_seqlens).to(dev)
+        B, s_q, H = inp.B, inp.s_q, inp.H
+        self.meta = torch.empty((mla.metadata_size(B, s_q, H) + 3) // 4, dtype=torch.int32, device=dev)
+        self.ws = torch.empty(mla.workspace_size(B, s_q, H), dtype=torch.uint8, device=dev)
+        self.out = torch.empty((B, s_q, H, 512), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((B, s_q, H), dtype=torch.float32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.stream = torch.cuda.current_stream()
+
+    def _step(self, ev=None):
+        m, i, st = self.mla, self.inp, self.stream
+        if ev is not None:
+            ev[0].record(st)
+        m.get_metadata(self.seqlens, i.s_q, i.H, metadata=self.meta, stream=st)
+        if ev is not None:
+            ev[1].record(st)
+        m.decode_attention(self.q_nope, self.q_pe, self.kv, self.table, self.seqlens, i.softmax_scale, i.causal,
+                           self.meta, self.ws, self.out, self.lse, status=self.status, stream=st)
+        if ev is not None:
+            ev[2].record(st)
+        m.decode_combine(self.seqlens, self.table.shape[1], i.s_q, i.H, self.meta, self.ws, self.out, self.lse,
+                         status=self.status, stream=st)
+        if ev is not None:
+            ev[3].record(st)
+
+    def steps(self, n, flush, timed=False):
+        """n steps with an L2 flush before each; with timed=True returns the summed
+        milliseconds of the step and of each launch (device events)."""
+        import torch
+
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)] if timed else None
+        for k in range(n):
+            flush()
+            self._step(evs[k] if timed else None)
+        if not timed:
+            return None
+        torch.cuda.synchronize()
+        tot = {"step": 0.0, "metadata": 0.0, "attention": 0.0, "combine": 0.0}
+        for e in evs:
+            tot["step"] += e[0].elapsed_time(e[3])
+            tot["metadata"] += e[0].elapsed_time(e[1])
+            tot["attention"] += e[1].elapsed_time(e[2])
+            tot["combine"] += e[2].elapsed_time(e[3])
+        return tot
+
+    def check_status(self, where):
+        v = int(self.status.item())
+        if v != 0:
+            raise RuntimeError(f"device status {v} in {where}")
+
+    def e2e(self, n):
+        """n steps through the public mla_decode call with pinned host inputs copied in
+        and out inside the timed region; returns (ms per step, H2D bytes, D2H bytes)."""
+        import torch
+
+        i, m, st = self.inp, self.mla, self.stream
+        h = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for k, v in
+             (("q_nope", i.q_nope.view(np.int16)), ("q_pe", i.q_pe.view(np.int16)),
+              ("kv", i.kv_cache.view(np.int16)), ("table", i.block_table), ("seq", i.cache_seqlens))}
+        h_out = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
+        h_lse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
+        d = {k: torch.empty(v.shape, dtype=v.dtype, device=self.dev) for k, v in h.items()}
+        h2d = sum(v.numel() * v.element_size() for v in h.values())
+        d2h = h_out.numel() * 2 + h_lse.numel() * 4
+
+        def one():
+            for k in h:
+                d[k].copy_(h[k], non_blocking=True)
+            meta = m.get_metadata(d["seq"], i.s_q, i.H, metadata=self.meta, stream=st)
+            m.decode(d["q_nope"].view(torch.bfloat16), d["q_pe"].view(torch.bfloat16), d["kv"].view(torch.bfloat16),
+                     d["table"], d["seq"], i.softmax_scale, i.causal, meta, workspace=self.ws, out=self.out,
+                     lse=self.lse, status=self.status, stream=st)
+            h_out.copy_(self.out, non_blocking=True)
+            h_lse.copy_(self.lse, non_blocking=True)
+
+        for _ in range(2):
+            one()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(n):
+            one()
+        e1.record(st)
+        torch.cuda.synchronize()
+        self.check_status("the end-to-end steps")
+        return e0.elapsed_time(e1) / n, h2d, d2h
+
+
+def roofline(inp, t, steps):
+    """Roofline figures of the attention kernel from summed device milliseconds.
+
+    Roofline time = max(cache bytes / HBM peak, FLOPs / bf16 peak); `achieved` is the
+    algorithmic bytes (HBM-bound) or FLOPs (tensor-bound) per launch over the kernel's
+    average duration; pct_of_roofline = roofline time / kernel time, and
+    pct_of_roofline_decode the same over the whole mla_decode call (attention +
+    combine)."""
+    hbm_peak, tc_peak, _, peak_src = load_peaks()
+    flops, cache_bytes, algo_bytes = algorithmic_work(inp.cache_seqlens, inp.s_q, inp.H, inp.causal)
+    att_s = t["attention"] / steps * 1e-3
+    t_hbm = cache_bytes / (hbm_peak * 1e9)
+    t_tc = flops / (tc_peak * 1e12)
+    if t_hbm >= t_tc:
+        achieved = algo_bytes / att_s / 1e9
+        r = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+             "peak_source": f"{peak_src} (burst copy)"}
+    else:
+        achieved = flops / att_s / 1e12
+        r = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s", "frac": achieved / tc_peak,
+             "peak_source": f"{peak_src} (burst bf16 GEMM)"}
+    r["kernel"] = "mla_decode_kernel (split-KV attention)"
+    r["kernel_avg_us"] = att_s * 1e6
+    r["roofline_us"] = max(t_hbm, t_tc) * 1e6
+    r["pct_of_roofline"] = max(t_hbm, t_tc) / att_s
+    r["step_us"] = t["step"] / steps * 1e3
+    r["step_without_metadata_us"] = (t["step"] - t["metadata"]) / steps * 1e3
+    r["pct_of_roofline_decode"] = max(t_hbm, t_tc) / ((t["attention"] + t["combine"]) / steps * 1e-3)
+    return r
+
+
+# ---------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -216,6 +382,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--per-workload-steps", type=int, default=30,
+                    help="timed steps for each of the other decode configurations (0 = skip)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -240,7 +408,7 @@ def main():
             nseq += n
         value = flops / secs / 1e12
         line = {
-            "impl": "reference", "metric": f"MLA decode TFLOP/s ({w.name})", "value": value, "unit": "TFLOP/s",
+            "impl": "reference", "metric": metric_name(w), "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "s_q": w.s_q, "H": w.H, "causal": w.causal,
@@ -265,134 +433,74 @@ def main():
     else:
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
+    flusher = L2Flush(dev)
 
     inp = make_workload(args.workload)
     flops, cache_bytes, algo_bytes = algorithmic_work(inp.cache_seqlens, inp.s_q, inp.H, inp.causal)
-
-    def to_dev_bf16(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
-
-    q_nope = to_dev_bf16(inp.q_nope)
-    q_pe = to_dev_bf16(inp.q_pe)
-    kv = to_dev_bf16(inp.kv_cache)
-    table = torch.from_numpy(inp.block_table).to(dev)
-    seqlens = torch.from_numpy(inp.cache_seqlens).to(dev)
     B, s_q, H = inp.B, inp.s_q, inp.H
-    meta = torch.empty((mla.metadata_size(B, s_q, H) + 3) // 4, dtype=torch.int32, device=dev)
-    ws = torch.empty(mla.workspace_size(B, s_q, H), dtype=torch.uint8, device=dev)
-    out = torch.empty((B, s_q, H, 512), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((B, s_q, H), dtype=torch.float32, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
+    run = DeviceRun(mla, inp, dev)
 
-    def step(ev=None):
-        mla.get_metadata(seqlens, s_q, H, metadata=meta, stream=stream)
-        if ev is not None:
-            ev[0].record(stream)
-        mla.decode_attention(q_nope, q_pe, kv, table, seqlens, inp.softmax_scale, inp.causal, meta, ws, out, lse,
-                             status=status, stream=stream)
-        if ev is not None:
-            ev[1].record(stream)
-        mla.decode_combine(seqlens, table.shape[1], s_q, H, meta, ws, out, lse, status=status, stream=stream)
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
+    run.steps(args.warmup, flusher)
     torch.cuda.synchronize()
-    if int(status.item()) != 0:
-        raise RuntimeError(f"device status {int(status.item())} during warm-up")
+    run.check_status("warm-up")
 
     K = args.steps
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(uuid)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with sampler:
-        for k in range(K):
-            flush.zero_()
-            ev_s[k].record(stream)
-            step(ev_a[k])
-            ev_e[k].record(stream)
+        t = run.steps(K, flusher, timed=True)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    step_ms = sum(ev_s[k].elapsed_time(ev_e[k]) for k in range(K))
-    att_ms = sum(ev_a[k][0].elapsed_time(ev_a[k][1]) for k in range(K))
-    if int(status.item()) != 0:
-        raise RuntimeError(f"device status {int(status.item())} in the timed region")
-    step_ms, att_ms = max_over_ranks([step_ms, att_ms], world, dev, dist)
+    run.check_status("the timed region")
+    step_ms, meta_ms, att_ms, comb_ms = max_over_ranks(
+        [t["step"], t["metadata"], t["attention"], t["combine"]], world, dev, dist)
 
     # ---- end to end through the public API with host buffers ---------------
     e2e = None
     if args.e2e_steps > 0:
-        h = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for k, v in
-             (("q_nope", inp.q_nope.view(np.int16)), ("q_pe", inp.q_pe.view(np.int16)),
-              ("kv", inp.kv_cache.view(np.int16)), ("table", inp.block_table), ("seq", inp.cache_seqlens))}
-        h_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
-        h_lse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
-        d = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in h.items()}
-        h2d = sum(v.numel() * v.element_size() for v in h.values())
-        d2h = h_out.numel() * 2 + h_lse.numel() * 4
-
-        def e2e_step():
-            for k in h:
-                d[k].copy_(h[k], non_blocking=True)
-            m = mla.get_metadata(d["seq"], s_q, H, metadata=meta, stream=stream)
-            mla.decode(d["q_nope"].view(torch.bfloat16), d["q_pe"].view(torch.bfloat16), d["kv"].view(torch.bfloat16),
-                       d["table"], d["seq"], inp.softmax_scale, inp.causal, m, workspace=ws, out=out, lse=lse,
-                       status=status, stream=stream)
-            h_out.copy_(out, non_blocking=True)
-            h_lse.copy_(lse, non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_ms, h2d, d2h = run.e2e(args.e2e_steps)
         if world > 1:
             dist.barrier()
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
         (e2e_ms,) = max_over_ranks([e2e_ms], world, dev, dist)
         e2e = {"value": whole_job_rate(world, flops, e2e_ms) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
+
+    # ---- the other decode configurations: attention-kernel figures ----------
+    per_workload = {}
+    if world == 1 and args.per_workload_steps > 0:
+        del run
+        torch.cuda.empty_cache()
+        for name in ("decode_b64", "mtp_b128_sq2", "serving_b256", "long_b4"):
+            if name == args.workload:
+                continue
+            wi = make_workload(name)
+            ri = DeviceRun(mla, wi, dev)
+            ri.steps(args.warmup, flusher)
+            ti = ri.steps(args.per_workload_steps, flusher, timed=True)
+            torch.cuda.synchronize()
+            ri.check_status(name)
+            per_workload[name] = roofline(wi, ti, args.per_workload_steps)
+            del ri
+            torch.cuda.empty_cache()
 
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
         return
 
-    hbm_peak, tc_peak, tc_sustained, peak_src = load_peaks()
     ms = step_ms / K
-    att_avg_s = att_ms / K * 1e-3
     value = whole_job_rate(world, flops, ms) / 1e12
-    t_hbm = cache_bytes / (hbm_peak * 1e9)
-    t_tc = flops / (tc_peak * 1e12)
-    bound = "hbm" if t_hbm >= t_tc else "tensor"
-    if bound == "hbm":
-        achieved = algo_bytes / att_avg_s / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                "traffic": recorded_traffic(w.name), "peak_source": peak_src + " (burst copy)"}
-    else:
-        achieved = flops / att_avg_s / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                "frac": achieved / tc_peak, "traffic": recorded_traffic(w.name),
-                "peak_source": peak_src + " (burst bf16 GEMM)"}
-    roof["kernel"] = "mla_decode_kernel (split-KV attention)"
-    roof["kernel_avg_us"] = att_avg_s * 1e6
-    roof["roofline_us"] = max(t_hbm, t_tc) * 1e6
-    roof["pct_of_roofline"] = max(t_hbm, t_tc) / att_avg_s
+    roof = roofline(inp, {"attention": att_ms, "step": step_ms, "metadata": meta_ms, "combine": comb_ms}, K)
+    per_workload[w.name] = {k: roof[k] for k in ("bound", "kernel_avg_us", "roofline_us", "pct_of_roofline", "frac",
+                                                 "step_us", "step_without_metadata_us", "pct_of_roofline_decode")}
+    roof["traffic"] = recorded_traffic(w.name)
 
     line = {
-        "metric": f"MLA decode TFLOP/s ({w.name}: B={B}, s_q={s_q}, H={H})",
+        "metric": metric_name(w),
         "value": value,
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -406,20 +514,24 @@ def main():
         "data": "synthetic",
         "config": {"workload": w.name, "B": B, "s_q": s_q, "H": H, "causal": w.causal, "lengths": w.lengths,
                    "seed": w.seed, "block_size": 64, "softmax_scale": inp.softmax_scale,
-                   "l2": "256 MB write before every step, outside the timed events",
+                   "l2": L2Flush.DESCRIPTION,
                    "parallelism": f"replicas x{world}"},
         "hbm_gbs": algo_bytes / (ms * 1e-3) / 1e9,
-        "kernel_tflops": flops / att_avg_s / 1e12,
+        "kernel_tflops": flops / (att_ms / K * 1e-3) / 1e12,
+        "metadata_us": meta_ms / K * 1e3,
+        "combine_us": comb_ms / K * 1e3,
+        "step_without_metadata_us": (step_ms - meta_ms) / K * 1e3,
         "roofline": roof,
+        "per_workload": per_workload,
         "gpu_launches": 3 * K,
         "clocks": sampler.summary(),
     }
     if e2e is not None:
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
-        f, s, n = time_oracle(inp, args.cpu_budget)
-        line["cpu_baseline"] = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-                                "sample": f"{n} whole sequences of {w.name} ({s:.1f} s, float64 numpy)"}
+        f, s_, n = time_oracle(inp, args.cpu_budget)
+        line["cpu_baseline"] = {"value": f / s_ / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                                "sample": f"{n} whole sequences of {w.name} ({s_:.1f} s, float64 numpy)"}
     print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()

@@ -10,8 +10,9 @@
 // Grid (P, ceil(M / 8)): block x = p looks at partition p's first block; a split
 // sequence is exactly one whose cut opens a partition mid-sequence, and the first such
 // partition (first_part + 1) owns its merge, so only blocks with work touch memory.
-// Rows of sequences that no partition covers (no visible key, invalid length) are
-// written by the attention kernel.
+// Rows of sequences that no partition covers (no visible key, invalid length, a block
+// count in the metadata that does not match the length) are written by the attention
+// kernel.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -38,7 +39,9 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
   if (b >= B || meta[off_part_start() + 2 * part + 1] == 0) return;  // partition opens a sequence
   if (meta[off_first_part(B) + b] + 1 != part) return;              // a later cut of the same sequence
   const int n = seqlens[b];
-  if (n < 0 || (int64_t)n > (int64_t)max_blocks * kBlockSize) return;  // rows written as NaN already
+  // rows written as NaN already: invalid length, or a schedule built for another length
+  if (n < 0 || (int64_t)n > (int64_t)max_blocks * kBlockSize) return;
+  if (meta[off_nblk() + b] != (n + kBlockSize - 1) / kBlockSize) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.y * kWarps + warp;
   if (row >= M) return;

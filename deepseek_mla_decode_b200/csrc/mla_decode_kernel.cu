@@ -107,8 +107,17 @@ struct Piece {
   int b, k_lo, k_hi, split, n;
 };
 
-// Walks the pieces of one partition.  Pieces of sequences whose length is invalid
-// are skipped consistently by every role (producer warp 0 writes their NaN rows).
+// Block count of a sequence of n keys, or -1 when n is not a valid length for the table.
+__device__ __forceinline__ int expected_blocks(const Params& p, int n) {
+  if (n < 0 || (int64_t)n > (int64_t)p.max_blocks * kBlockSize) return -1;
+  return (n + kBlockSize - 1) / kBlockSize;
+}
+
+// Walks the pieces of one partition.  Pieces of sequences whose length is invalid, or
+// whose block count in the metadata is not the one their current length needs (a
+// schedule built for other lengths), are skipped consistently by every role (producer
+// warp 0 writes their NaN rows).  Piece bounds are clamped to the sequence's blocks, so
+// no block-table entry past ceil(n / 64) is ever read.
 struct PieceWalker {
   const Params* p;
   int cb, ck, be, ke;
@@ -125,14 +134,16 @@ struct PieceWalker {
     first_part = m + off_first_part(prm.B);
   }
   __device__ bool next(Piece& pc) {
+    if (cb < 0) cb = p->B;  // malformed start: no pieces
     while (cb < p->B && (cb < be || (cb == be && ck < ke))) {
-      const int hi = (cb == be) ? ke : nblk[cb];
-      const int b = cb, lo = ck;
+      const int nb = nblk[cb];
+      const int hi = min((cb == be) ? ke : nb, nb);
+      const int b = cb, lo = max(ck, 0);
       cb += 1;
       ck = 0;
       if (lo >= hi) continue;
       const int n = p->seqlens[b];
-      if (n < 0 || (int64_t)n > (int64_t)p->max_blocks * kBlockSize) continue;
+      if (expected_blocks(*p, n) != nb) continue;
       pc.b = b;
       pc.k_lo = lo;
       pc.k_hi = hi;
@@ -272,15 +283,21 @@ __device__ __forceinline__ int clamp_block_id(const Params& p, int32_t id) {
   return id;
 }
 
-// Rows of sequences that no partition covers: no visible key (out 0, lse -inf) or an
-// invalid length (NaN and the status bit).  Partition `part` takes the sequences b with
-// b % P == part; the 32 lanes of one warp write this CTA's 64 rows [y0, y0 + 64).
+// Rows of sequences that no partition covers: no visible key (out 0, lse -inf), an
+// invalid length (NaN and MLA_DEVICE_ERR_SEQLEN) or a block count in the metadata that
+// does not match the current length (NaN and MLA_DEVICE_ERR_METADATA).  Partition `part`
+// takes the sequences b with b % P == part; the 32 lanes of one warp write this CTA's
+// 64 rows [y0, y0 + 64).
 __device__ __forceinline__ void write_orphan_rows(const Params& p, int part, int P, int y0, int lane) {
+  const int32_t* nblk = p.meta + off_nblk();
   for (int b = part; b < p.B; b += P) {
     const int n = p.seqlens[b];
-    const bool bad_len = n < 0 || (int64_t)n > (int64_t)p.max_blocks * kBlockSize;
-    if (!bad_len && n > 0) continue;
-    const float v = bad_len ? __int_as_float(0x7fc00000) : 0.0f;
+    const int want = expected_blocks(p, n);
+    const bool bad_len = want < 0;
+    const bool stale = !bad_len && nblk[b] != want;
+    if (!bad_len && !stale && n > 0) continue;
+    const bool bad = bad_len || stale;
+    const float v = bad ? __int_as_float(0x7fc00000) : 0.0f;
     const uint32_t pv = pack_bf16x2(v, v);
     for (int i = lane; i < kRowsPerCta * (kDLatent / 8); i += 32) {  // 16-byte units
       const int row = y0 + i / (kDLatent / 8);
@@ -289,8 +306,8 @@ __device__ __forceinline__ void write_orphan_rows(const Params& p, int part, int
             make_uint4(pv, pv, pv, pv);
     }
     for (int r = lane; r < kRowsPerCta; r += 32)
-      if (y0 + r < p.M) p.lse[(int64_t)b * p.M + y0 + r] = bad_len ? __int_as_float(0x7fc00000) : -INFINITY;
-    if (bad_len && lane == 0) set_status(p, kErrSeqlen);
+      if (y0 + r < p.M) p.lse[(int64_t)b * p.M + y0 + r] = bad ? __int_as_float(0x7fc00000) : -INFINITY;
+    if (bad && lane == 0) set_status(p, bad_len ? kErrSeqlen : kErrMetadata);
   }
 }
 

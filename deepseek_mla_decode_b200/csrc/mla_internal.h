@@ -33,7 +33,7 @@ enum HdrField : int {
   kHdrH = 3,
   kHdrNumParts = 4,   // P: partitions per row tile
   kHdrNumTiles = 5,   // T: row tiles of 128 query rows
-  kHdrCap = 6,        // partition cost cap (blocks)
+  kHdrCap = 6,        // partition cost cap (256-key tiles)
   kHdrTotalSlots = 7, // sum of num_splits
   kHdrNumWorkers = 8, // CTA pairs available on the device
   kHdrOverhead = 9,

@@ -29,10 +29,12 @@
  *  - Calls that take a stream are asynchronous on that stream.  Host-detectable
  *    errors are returned before anything is launched; nothing else is written.
  *  - Device-detectable data errors (a block id outside [0, num_blocks) among the
- *    blocks a sequence uses, n_b < 0, n_b > max_blocks * 64) never fault: the
- *    affected sequence's out rows and lse are set to NaN and a bit is OR-ed into
- *    *status (MLA_DEVICE_ERR_*) when status != NULL.  A bounded wait inside a
- *    kernel that runs out (1 s) sets MLA_DEVICE_ERR_TIMEOUT and the kernel returns.
+ *    blocks a sequence uses, n_b < 0, n_b > max_blocks * 64, metadata whose block
+ *    count for a sequence is not ceil(n_b / 64)) never fault and never read past a
+ *    sequence's blocks: the affected sequence's out rows and lse are set to NaN and
+ *    a bit is OR-ed into *status (MLA_DEVICE_ERR_*) when status != NULL.  A bounded
+ *    wait inside a kernel that runs out (1 s) sets MLA_DEVICE_ERR_TIMEOUT and the
+ *    kernel returns.
  *  - No C++ exception crosses this boundary.  Calls are re-entrant given distinct
  *    metadata / workspace buffers.
  */
@@ -59,7 +61,9 @@ typedef enum {
 #define MLA_DEVICE_ERR_BLOCK_ID 1 /* block_table entry outside [0, num_blocks) */
 #define MLA_DEVICE_ERR_SEQLEN 2   /* cache_seqlens[b] < 0 or > max_blocks * 64  */
 #define MLA_DEVICE_ERR_TIMEOUT 4  /* an internal bounded wait ran out           */
-#define MLA_DEVICE_ERR_METADATA 8 /* metadata not produced for these B, s_q, H   */
+#define MLA_DEVICE_ERR_METADATA 8 /* metadata not produced for these B, s_q, H, or
+                                     for another length of some sequence (its block
+                                     count differs; that sequence's rows are NaN)   */
 
 /* Fixed geometry. */
 #define MLA_BLOCK_SIZE 64  /* cache rows per physical block   */
@@ -74,7 +78,8 @@ const char* mla_status_string(mla_status_t status);
 
 /*
  * Bytes of the schedule buffer mla_get_metadata writes for (B, s_q, H).  Host only,
- * no device call.  *bytes receives the size.
+ * no device call.  *bytes receives the size.  Library convenience: no passage of the
+ * source pages corresponds to it.
  */
 mla_status_t mla_metadata_size(int B, int s_q, int H, size_t* bytes);
 
@@ -99,6 +104,8 @@ mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int B, int s_q, int 
 /*
  * Upper bound, in bytes, of the fp32 scratch mla_decode needs for split partial
  * results (partial outputs and their lse) for (B, s_q, H) on the current device.
+ * The partials are the split-K intermediate results of the "DeepSeek speed test /
+ * FA3" article, section 2.1; the size query itself is a library convenience.
  */
 mla_status_t mla_workspace_size(int B, int s_q, int H, size_t* bytes);
 
@@ -136,11 +143,15 @@ mla_status_t mla_decode(const void* q_nope, const void* q_pe, const void* kv_cac
  * semantics; mla_decode == mla_decode_attention followed by mla_decode_combine on
  * the same stream with the same workspace).
  *
- * mla_decode_attention: the split-KV attention kernel.  Sequences processed in one
- *   piece get their out / lse rows written directly; pieces of split sequences write
- *   normalised fp32 partial outputs and their lse into the workspace.  It also writes
- *   the rows of sequences with no visible key (0 / -inf) and of sequences with an
- *   invalid length (NaN, MLA_DEVICE_ERR_SEQLEN).
+ * mla_decode_attention: the split-KV attention kernel (the
+ *   weight-absorbed attention of the KsanaLLM 0.6.0 release notes, section 2.1, with
+ *   the split-K partials of the "DeepSeek speed test / FA3" article, section 2.1).
+ *   Sequences processed in one piece get their out / lse rows written directly;
+ *   pieces of split sequences write normalised fp32 partial outputs and their lse into
+ *   the workspace.  It also writes the rows of sequences with no visible key
+ *   (0 / -inf) and of sequences with an invalid length (NaN, MLA_DEVICE_ERR_SEQLEN)
+ *   or a stale block count in the metadata (NaN, MLA_DEVICE_ERR_METADATA).  Exposing
+ *   it separately is a library convenience (timing, custom merges).
  * mla_decode_combine: the LSE-combine kernel (split-K merge, "DeepSeek speed test /
  *   FA3" article section 2.1): for every split sequence, lse = ln sum_s exp(lse_s) and
  *   out = sum_s exp(lse_s - lse) O_s.  Only split sequences are touched; `status` is
@@ -185,7 +196,8 @@ mla_status_t mla_decode_noalloc(const void* q_nope, const void* q_pe, const void
                                 size_t metadata_bytes, void* out, float* lse, int32_t* status,
                                 void* stream);
 
-/* Number of streaming multiprocessors the schedule targets on the current device. */
+/* Number of streaming multiprocessors the schedule targets on the current device.
+ * Library convenience: no passage of the source pages corresponds to it. */
 mla_status_t mla_device_sm_count(int* sm_count);
 
 #ifdef __cplusplus
