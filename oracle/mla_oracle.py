@@ -97,6 +97,7 @@ def mla_decode_ref(
     cache_seqlens: np.ndarray,
     softmax_scale: float,
     causal: bool,
+    q_lens=None,
 ) -> Tuple[np.ndarray, np.ndarray]:
     """Weight-absorbed MLA decode attention, float64, no tiling or online softmax.
 
@@ -107,6 +108,13 @@ def mla_decode_ref(
         s_t   = scale * (q_nope . c_kv[t] + q_pe . k_pe[t])   for visible t
         lse   = ln sum_t exp(s_t)            (computed as m + ln sum exp(s_t - m))
         out   = sum_t exp(s_t - lse) * c_kv[t]
+
+    ``q_lens`` [B] (optional) gives sequence b its own number of query tokens
+    q_lens[b] <= s_q (draft tokens accepted per sequence differ in speculative
+    decoding: Paddle 3.0 article, speculative-decoding section).  Its new tokens are
+    the last q_lens[b] cache positions, so with the causal mask token i sees keys
+    0 .. n - q_lens[b] + i; tokens i >= q_lens[b] are padding and give out = 0,
+    lse = -inf.  Without q_lens every sequence has s_q tokens.
     """
     B, s_q, H, dl = q_nope.shape
     assert dl == D_LATENT and q_pe.shape == (B, s_q, H, D_ROPE)
@@ -115,11 +123,13 @@ def mla_decode_ref(
     lse = np.full((B, s_q, H), -np.inf, dtype=np.float64)
     for b in range(B):
         n = int(cache_seqlens[b])
+        s_b = s_q if q_lens is None else int(q_lens[b])
+        assert 0 <= s_b <= s_q
         rows = gather_rows(kv_cache, block_table[b], n)  # [n, 576]
         q = np.concatenate([q_nope[b], q_pe[b]], axis=-1)  # [s_q, H, 576]
         scores = softmax_scale * (q @ rows.T)  # [s_q, H, n]
-        for i in range(s_q):
-            nv = visible_key_count(n, s_q, i, causal)
+        for i in range(s_b):
+            nv = visible_key_count(n, s_b, i, causal)
             if nv == 0:
                 continue  # out stays 0, lse stays -inf
             s = scores[i, :, :nv]

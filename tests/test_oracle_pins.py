@@ -211,6 +211,31 @@ def test_causal_sq2_equals_two_sq1_calls():
         assert np.array_equal(out[:, i], o1[:, 0]) and np.array_equal(lse[:, i], l1[:, 0])
 
 
+def test_ragged_query_counts_equal_single_token_calls():
+    """Per-sequence query counts: token i of sequence b with q_lens[b] = L, causal,
+    over n keys == an s_q = 1 call over n - L + i + 1 keys (bit-exact); tokens
+    i >= L are padding (out 0, lse -inf); q_lens = s_q everywhere is the uniform call."""
+    inp = make_inputs(4, 4, 6, [3, 70, 300, 9], seed=23, causal=True)
+    qn, qp, kv = f64(inp)
+    q_lens = np.array([2, 4, 1, 0])
+    out, lse = O.mla_decode_ref(qn, qp, kv, inp.block_table, inp.cache_seqlens, inp.softmax_scale, True,
+                                q_lens=q_lens)
+    for b in range(inp.B):
+        L, n = int(q_lens[b]), int(inp.cache_seqlens[b])
+        for i in range(4):
+            if i >= L:
+                assert np.all(out[b, i] == 0) and np.all(np.isneginf(lse[b, i]))
+                continue
+            o1, l1 = O.mla_decode_ref(qn[b : b + 1, i : i + 1], qp[b : b + 1, i : i + 1], kv,
+                                      inp.block_table[b : b + 1], np.array([n - L + i + 1]), inp.softmax_scale,
+                                      False)
+            assert np.array_equal(out[b, i], o1[0, 0]) and np.array_equal(lse[b, i], l1[0, 0])
+    u = O.mla_decode_ref(qn, qp, kv, inp.block_table, inp.cache_seqlens, inp.softmax_scale, True,
+                         q_lens=np.full(4, 4))
+    v = O.mla_decode_ref(qn, qp, kv, inp.block_table, inp.cache_seqlens, inp.softmax_scale, True)
+    assert np.array_equal(u[0], v[0]) and np.array_equal(u[1], v[1])
+
+
 def test_causal_sq1_equals_noncausal():
     inp = make_inputs(2, 1, 4, [5, 99], seed=18)
     a = run(inp, causal=True)
