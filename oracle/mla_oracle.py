@@ -142,6 +142,32 @@ def mla_decode_ref(
 
 
 # ----------------------------------------------------------------------------
+# weight absorption either side of the decode
+# ----------------------------------------------------------------------------
+D_NOPE = 128  # per-head no-RoPE query / value width of DeepSeek's attention head
+
+
+def absorb_q_ref(q_heads: np.ndarray, w_uk: np.ndarray) -> np.ndarray:
+    """Absorbed latent query: q_nope[b,i,h,:] = W_UK[h]^T q[b,i,h,:].
+
+    q_heads [B, s_q, H, 128] (the per-head no-RoPE queries), w_uk [H, 128, 512] (the
+    key up-projection of each head, k_h = W_UK[h] c).  Folding W_UK into the query
+    lets every head score the shared 512-d latent directly (KsanaLLM 0.6.0 release
+    notes, section 2.1, WA-MLA).  Returns [B, s_q, H, 512], float64."""
+    return np.einsum("bihd,hdc->bihc", q_heads, w_uk)
+
+
+def absorb_out_ref(o_latent: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
+    """Per-head output from the latent one: y[b,i,h,:] = W_UV[h] o[b,i,h,:].
+
+    o_latent [B, s_q, H, 512] (the decode output), w_uv [H, 128, 512] (the value
+    up-projection of each head, v_h = W_UV[h] c); the attention-weighted sum of
+    v_h is W_UV[h] applied to the weighted sum of latents (same section).  Returns
+    [B, s_q, H, 128], float64."""
+    return np.einsum("bihc,hdc->bihd", o_latent, w_uv)
+
+
+# ----------------------------------------------------------------------------
 # split-KV partials and their log-sum-exp merge
 # ----------------------------------------------------------------------------
 def partial_ref(

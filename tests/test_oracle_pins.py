@@ -89,6 +89,34 @@ def test_equals_nonabsorbed_mla():
     assert np.max(np.abs(lse_abs[0, 0] - lse_full)) < 1e-12
 
 
+def test_absorption_gemms_equal_nonabsorbed_mla():
+    """absorb_q_ref -> mla_decode_ref -> absorb_out_ref equals textbook attention
+    with explicit per-head keys [W_UK c ; k_pe] and values W_UV c (to 1e-12), on a
+    paged batch with two query tokens, causal."""
+    rng = np.random.default_rng(6)
+    inp = make_inputs(2, 2, 4, [9, 70], seed=24, causal=True)
+    qn_lat, qp, kv = f64(inp)
+    q_h = rng.standard_normal((2, 2, 4, 128))
+    W_UK = rng.standard_normal((4, 128, 512)) * 0.05
+    W_UV = rng.standard_normal((4, 128, 512)) * 0.05
+    q_abs = O.absorb_q_ref(q_h, W_UK)
+    out_lat, lse = O.mla_decode_ref(q_abs, qp, kv, inp.block_table, inp.cache_seqlens, inp.softmax_scale, True)
+    y = O.absorb_out_ref(out_lat, W_UV)
+    for b in range(2):
+        n = int(inp.cache_seqlens[b])
+        rows = O.gather_rows(kv, inp.block_table[b], n)
+        c, k_pe = rows[:, :512], rows[:, 512:]
+        for i in range(2):
+            nv = n - 2 + i + 1
+            for h in range(4):
+                K = np.concatenate([c[:nv] @ W_UK[h].T, k_pe[:nv]], axis=1)
+                V = c[:nv] @ W_UV[h].T
+                sc = inp.softmax_scale * K @ np.concatenate([q_h[b, i, h], qp[b, i, h]])
+                w = np.exp(sc - sc.max())
+                assert np.max(np.abs((w / w.sum()) @ V - y[b, i, h])) < 1e-12
+                assert abs(sc.max() + math.log(w.sum()) - lse[b, i, h]) < 1e-12
+
+
 # ---------------------------------------------------------------------------
 # closed forms
 # ---------------------------------------------------------------------------
