@@ -235,7 +235,7 @@ class L2Flush:
         import torch
 
         self.w.zero_()
-        torch.sum(self.r, out=self.sink)
+        torch.sum(self.r, dim=0, out=self.sink)
 
 
 class DeviceRun:

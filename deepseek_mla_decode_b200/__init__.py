@@ -30,10 +30,15 @@ EXPORTED_SYMBOLS = (
     "mla_get_metadata",
     "mla_workspace_size",
     "mla_decode",
+    "mla_decode_ragged",
     "mla_decode_attention",
     "mla_decode_combine",
     "mla_decode_noalloc",
     "mla_device_sm_count",
+    "mla_set_wait_timeout_ns",
+    "mla_set_stall_injection",
+    "mla_absorb_q",
+    "mla_absorb_out",
 )
 
 _lib = None
@@ -68,6 +73,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.mla_workspace_size.argtypes = [c_int, c_int, c_int, ctypes.POINTER(c_size)]
     L.mla_device_sm_count.restype = c_int
     L.mla_device_sm_count.argtypes = [ctypes.POINTER(c_int)]
+    L.mla_set_wait_timeout_ns.restype = c_int
+    L.mla_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+    L.mla_set_stall_injection.restype = c_int
+    L.mla_set_stall_injection.argtypes = [c_int]
     L.mla_get_metadata.restype = c_int
     L.mla_get_metadata.argtypes = [c_vp, c_int, c_int, c_int, c_vp, c_size, c_vp]
     dec_args = [c_vp, c_vp, c_vp, c_i64, c_vp, c_int, c_vp, c_int, c_int, c_int, c_f, c_int,
@@ -75,6 +84,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for fn in (L.mla_decode, L.mla_decode_attention):
         fn.restype = c_int
         fn.argtypes = dec_args
+    L.mla_decode_ragged.restype = c_int
+    L.mla_decode_ragged.argtypes = dec_args[:7] + [c_vp] + dec_args[7:]
+    for fn in (L.mla_absorb_q, L.mla_absorb_out):
+        fn.restype = c_int
+        fn.argtypes = [c_vp, c_vp, c_vp, c_int, c_int, c_vp]
     L.mla_decode_noalloc.restype = c_int
     L.mla_decode_noalloc.argtypes = [c_vp, c_vp, c_vp, c_i64, c_vp, c_int, c_vp, c_int, c_int, c_int, c_f, c_int,
                                      c_vp, c_size, c_vp, c_vp, c_vp, c_vp]
@@ -110,6 +124,18 @@ def device_sm_count() -> int:
     n = ctypes.c_int()
     _check("mla_device_sm_count", load_library().mla_device_sm_count(ctypes.byref(n)))
     return n.value
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    """Bound on the attention kernel's internal waits for later launches (0 = the
+    default 1 s); see mla_set_wait_timeout_ns."""
+    _check("mla_set_wait_timeout_ns", load_library().mla_set_wait_timeout_ns(int(ns)))
+
+
+def set_stall_injection(enable: bool) -> None:
+    """Test hook: make later launches' MMA warp wait on a barrier nothing completes,
+    so the bounded waits run out (see mla_set_stall_injection)."""
+    _check("mla_set_stall_injection", load_library().mla_set_stall_injection(int(bool(enable))))
 
 
 def _stream_ptr(stream) -> int:
@@ -168,6 +194,55 @@ def decode(q_nope, q_pe, kv_cache, block_table, cache_seqlens, softmax_scale: fl
         *_decode_args(q_nope, q_pe, kv_cache, block_table, cache_seqlens, softmax_scale, causal, metadata,
                       workspace, out, lse, status, stream)))
     return out, lse
+
+
+def decode_ragged(q_nope, q_pe, kv_cache, block_table, cache_seqlens, q_lens, softmax_scale: float, causal: bool,
+                  metadata, workspace=None, out=None, lse=None, status=None, stream=None) -> Tuple[object, object]:
+    """mla_decode_ragged: the decode with q_lens[b] <= s_q query tokens for sequence b
+    (padding tokens give out 0, lse -inf)."""
+    workspace, out, lse = _alloc_outputs(q_nope, workspace, out, lse)
+    if not q_lens.is_contiguous():
+        raise ValueError("q_lens must be contiguous")
+    args = _decode_args(q_nope, q_pe, kv_cache, block_table, cache_seqlens, softmax_scale, causal, metadata,
+                        workspace, out, lse, status, stream)
+    _check("mla_decode_ragged", load_library().mla_decode_ragged(*args[:7], q_lens.data_ptr(), *args[7:]))
+    return out, lse
+
+
+def absorb_q(q_heads, w_uk, q_nope=None, stream=None):
+    """mla_absorb_q: q_nope[..., h, :] = W_UK[h]^T q_heads[..., h, :] for q_heads
+    [B, s_q, H, 128] and w_uk [H, 128, 512]; returns q_nope [B, s_q, H, 512] (bf16)."""
+    import torch
+
+    *lead, H, d = q_heads.shape
+    if d != 128 or tuple(w_uk.shape) != (H, 128, 512):
+        raise ValueError("q_heads [..., H, 128] and w_uk [H, 128, 512] expected")
+    if not (q_heads.is_contiguous() and w_uk.is_contiguous()):
+        raise ValueError("inputs must be contiguous")
+    R = q_heads.numel() // (H * 128)
+    if q_nope is None:
+        q_nope = torch.empty((*lead, H, 512), dtype=torch.bfloat16, device=q_heads.device)
+    _check("mla_absorb_q", load_library().mla_absorb_q(q_heads.data_ptr(), w_uk.data_ptr(), q_nope.data_ptr(), R, H,
+                                                       _stream_ptr(stream)))
+    return q_nope
+
+
+def absorb_out(o_latent, w_uv, y=None, stream=None):
+    """mla_absorb_out: y[..., h, :] = W_UV[h] o_latent[..., h, :] for o_latent
+    [B, s_q, H, 512] and w_uv [H, 128, 512]; returns y [B, s_q, H, 128] (bf16)."""
+    import torch
+
+    *lead, H, d = o_latent.shape
+    if d != 512 or tuple(w_uv.shape) != (H, 128, 512):
+        raise ValueError("o_latent [..., H, 512] and w_uv [H, 128, 512] expected")
+    if not (o_latent.is_contiguous() and w_uv.is_contiguous()):
+        raise ValueError("inputs must be contiguous")
+    R = o_latent.numel() // (H * 512)
+    if y is None:
+        y = torch.empty((*lead, H, 128), dtype=torch.bfloat16, device=o_latent.device)
+    _check("mla_absorb_out", load_library().mla_absorb_out(o_latent.data_ptr(), w_uv.data_ptr(), y.data_ptr(), R, H,
+                                                           _stream_ptr(stream)))
+    return y
 
 
 def decode_attention(q_nope, q_pe, kv_cache, block_table, cache_seqlens, softmax_scale: float, causal: bool,

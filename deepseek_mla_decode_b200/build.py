@@ -18,7 +18,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmla.so")
-SOURCES = ["mla_api.cu", "mla_metadata.cu", "mla_decode_kernel.cu", "mla_combine.cu", "mla_noalloc.cu"]
+SOURCES = ["mla_api.cu", "mla_metadata.cu", "mla_decode_kernel.cu", "mla_combine.cu", "mla_noalloc.cu",
+           "mla_absorb.cu"]
 HEADERS = ["mla_internal.h", "ptx_sm100.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include "mla_internal.h"
 #include "../../include/mla_decode.h"
@@ -12,17 +13,18 @@
 namespace mla {
 cudaError_t launch_metadata(const int32_t* seqlens, int B, int s_q, int H, int num_workers, int32_t* meta,
                             cudaStream_t stream);
-cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, int max_blocks, int B, int M, int P,
-                           const float* part_o, const float* part_lse, void* out, float* lse,
-                           cudaStream_t stream);
+cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, const int32_t* q_lens, int max_blocks,
+                           int B, int s_q, int M, int P, const float* part_o, const float* part_lse, void* out,
+                           float* lse, cudaStream_t stream);
 cudaError_t decode_kernel_setup(int device);
 cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
                           const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
                           const CUtensorMap& tm_out, const CUtensorMap& tm_part,
                           const int32_t* block_table, int max_blocks, const int32_t* seqlens,
-                          const int32_t* meta, int64_t num_blocks, int B, int s_q, int H, float scale,
-                          int causal, void* out, float* lse, float* part_o, float* part_lse,
-                          int32_t* status, int num_ctas, cudaStream_t stream);
+                          const int32_t* q_lens, const int32_t* meta, int64_t num_blocks, int B, int s_q,
+                          int H, float scale, int causal, void* out, float* lse, float* part_o, float* part_lse,
+                          int32_t* status, int num_ctas, uint64_t wait_timeout_ns, int inject_stall,
+                          cudaStream_t stream);
 }  // namespace mla
 
 namespace {
@@ -41,6 +43,9 @@ struct DeviceInfo {
 
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
+constexpr uint64_t kDefaultWaitTimeoutNs = 1000000000ull;  // 1 s
+std::atomic<uint64_t> g_wait_timeout_ns{kDefaultWaitTimeoutNs};
+std::atomic<int> g_inject_stall{0};
 EncodeTiledFn g_encode = nullptr;
 
 // Per-device one-time setup: SM count, architecture check, kernel attributes.
@@ -105,6 +110,15 @@ bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, 
 
 }  // namespace
 
+namespace mla {
+// bf16 tiled tensor map with the 128-byte swizzle (the device must have been checked
+// with device_info first, which resolves the driver entry point)
+bool encode_tiled_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                       const cuuint32_t* box) {
+  return g_encode != nullptr && encode(m, base, rank, dims, strides, box);
+}
+}  // namespace mla
+
 extern "C" {
 
 const char* mla_status_string(mla_status_t s) {
@@ -123,6 +137,16 @@ mla_status_t mla_metadata_size(int B, int s_q, int H, size_t* bytes) {
   if (!bytes) return MLA_ERR_INVALID_ARG;
   if (!shape_supported(B, s_q, H)) return MLA_ERR_UNSUPPORTED;
   *bytes = static_cast<size_t>(mla::meta_words(B)) * sizeof(int32_t);
+  return MLA_OK;
+}
+
+mla_status_t mla_set_wait_timeout_ns(uint64_t ns) {
+  g_wait_timeout_ns.store(ns == 0 ? kDefaultWaitTimeoutNs : ns);
+  return MLA_OK;
+}
+
+mla_status_t mla_set_stall_injection(int enable) {
+  g_inject_stall.store(enable ? 1 : 0);
   return MLA_OK;
 }
 
@@ -202,8 +226,9 @@ mla_status_t check_decode_args(const void* q_nope, const void* q_pe, const void*
 }
 
 mla_status_t launch_attention(const void* q_nope, const void* q_pe, const void* kv_cache, int64_t num_blocks,
-                              const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens, int B,
-                              int s_q, int H, float softmax_scale, int causal, const void* metadata,
+                              const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                              const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
+                              const void* metadata,
                               void* workspace, void* out, float* lse, int32_t* status, const DecodeGeom& g,
                               cudaStream_t s) {
   const int64_t rows = static_cast<int64_t>(B) * g.M;
@@ -253,8 +278,9 @@ mla_status_t launch_attention(const void* q_nope, const void* q_pe, const void* 
       return MLA_ERR_INVALID_ARG;
   }
   if (mla::launch_decode(tm_kv, tm_kv2, tm_qn, tm_qp, tm_out, tm_part, block_table, max_blocks, cache_seqlens,
-                         static_cast<const int32_t*>(metadata), num_blocks, B, s_q, H, softmax_scale, causal != 0,
-                         out, lse, part_o, part_lse, status, 2 * g.P * g.T, s) != cudaSuccess)
+                         q_lens, static_cast<const int32_t*>(metadata), num_blocks, B, s_q, H, softmax_scale,
+                         causal != 0,
+                         out, lse, part_o, part_lse, status, 2 * g.P * g.T, g_wait_timeout_ns.load(), g_inject_stall.load(), s) != cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;
 }
@@ -273,8 +299,8 @@ mla_status_t mla_decode_attention(const void* q_nope, const void* q_pe, const vo
                                       B, s_q, H, softmax_scale, metadata, metadata_bytes, workspace,
                                       workspace_bytes, out, lse, status, &g);
   if (st != MLA_OK) return st;
-  return launch_attention(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, B, s_q, H,
-                          softmax_scale, causal, metadata, workspace, out, lse, status, g,
+  return launch_attention(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, nullptr, B,
+                          s_q, H, softmax_scale, causal, metadata, workspace, out, lse, status, g,
                           static_cast<cudaStream_t>(stream));
 }
 
@@ -301,7 +327,7 @@ mla_status_t mla_decode_combine(const int32_t* cache_seqlens, int max_blocks, in
   const float* part_o = static_cast<const float*>(workspace);
   const float* part_lse = part_o + slots * M * mla::kDLatent;
   (void)status;  // the combine raises no error of its own
-  if (mla::launch_combine(static_cast<const int32_t*>(metadata), cache_seqlens, max_blocks, B, M,
+  if (mla::launch_combine(static_cast<const int32_t*>(metadata), cache_seqlens, nullptr, max_blocks, B, s_q, M,
                           parts_for(num_workers_for(sms), s_q, H), part_o, part_lse, out, lse,
                           static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MLA_ERR_CUDA;
@@ -313,19 +339,30 @@ mla_status_t mla_decode(const void* q_nope, const void* q_pe, const void* kv_cac
                         int s_q, int H, float softmax_scale, int causal, const void* metadata,
                         size_t metadata_bytes, void* workspace, size_t workspace_bytes, void* out, float* lse,
                         int32_t* status, void* stream) {
+  return mla_decode_ragged(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, nullptr, B,
+                           s_q, H, softmax_scale, causal, metadata, metadata_bytes, workspace, workspace_bytes, out,
+                           lse, status, stream);
+}
+
+mla_status_t mla_decode_ragged(const void* q_nope, const void* q_pe, const void* kv_cache, int64_t num_blocks,
+                               const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                               const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
+                               const void* metadata, size_t metadata_bytes, void* workspace,
+                               size_t workspace_bytes, void* out, float* lse, int32_t* status, void* stream) {
+  if (q_lens && (reinterpret_cast<uintptr_t>(q_lens) & 3u)) return MLA_ERR_INVALID_ARG;
   DecodeGeom g;
   mla_status_t st = check_decode_args(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens,
                                       B, s_q, H, softmax_scale, metadata, metadata_bytes, workspace,
                                       workspace_bytes, out, lse, status, &g);
   if (st != MLA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_attention(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, B, s_q, H,
-                        softmax_scale, causal, metadata, workspace, out, lse, status, g, s);
+  st = launch_attention(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, q_lens, B, s_q,
+                        H, softmax_scale, causal, metadata, workspace, out, lse, status, g, s);
   if (st != MLA_OK) return st;
   const float* part_o = static_cast<const float*>(workspace);
   const float* part_lse = part_o + g.slots * g.M * mla::kDLatent;
-  if (mla::launch_combine(static_cast<const int32_t*>(metadata), cache_seqlens, max_blocks, B, g.M, g.P, part_o,
-                          part_lse, out, lse, s) != cudaSuccess)
+  if (mla::launch_combine(static_cast<const int32_t*>(metadata), cache_seqlens, q_lens, max_blocks, B, s_q, g.M,
+                          g.P, part_o, part_lse, out, lse, s) != cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;
 }

@@ -30,8 +30,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 }
 
 __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
-    const int32_t* __restrict__ meta, const int32_t* __restrict__ seqlens, int max_blocks,
-    int B, int M, const float* __restrict__ part_o, const float* __restrict__ part_lse,
+    const int32_t* __restrict__ meta, const int32_t* __restrict__ seqlens, const int32_t* __restrict__ q_lens,
+    int max_blocks, int B, int s_q, int M, const float* __restrict__ part_o, const float* __restrict__ part_lse,
     __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
   const int part = blockIdx.x;
   if (part == 0) return;
@@ -42,9 +42,13 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
   // rows written as NaN already: invalid length, or a schedule built for another length
   if (n < 0 || (int64_t)n > (int64_t)max_blocks * kBlockSize) return;
   if (meta[off_nblk() + b] != (n + kBlockSize - 1) / kBlockSize) return;
+  const int ql = q_lens ? q_lens[b] : s_q;
+  if (ql < 0 || ql > s_q) return;  // invalid query count: NaN rows written already
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.y * kWarps + warp;
   if (row >= M) return;
+  // a row tile holding only padding tokens had no pieces; its rows are written already
+  if ((row / kRowsPerTile) * kRowsPerTile >= ql * (M / s_q)) return;
   const int ns = meta[off_num_splits(B) + b];
   uint2* orow = reinterpret_cast<uint2*>(out + ((int64_t)b * M + row) * kDLatent);
   const int64_t slot0 = meta[off_split_prefix(B) + b];
@@ -91,11 +95,11 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
 
 }  // namespace
 
-cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, int max_blocks, int B,
-                           int M, int P, const float* part_o, const float* part_lse, void* out, float* lse,
+cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, const int32_t* q_lens, int max_blocks,
+                           int B, int s_q, int M, int P, const float* part_o, const float* part_lse, void* out, float* lse,
                            cudaStream_t stream) {
   dim3 grid(P, (M + kWarps - 1) / kWarps);
-  combine_kernel<<<grid, kWarps * 32, 0, stream>>>(meta, seqlens, max_blocks, B, M, part_o, part_lse,
+  combine_kernel<<<grid, kWarps * 32, 0, stream>>>(meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o, part_lse,
                                                    reinterpret_cast<__nv_bfloat16*>(out), lse);
   return cudaGetLastError();
 }

@@ -23,9 +23,10 @@
 // producer k % 4), warp 1 = MMA issuer (leader CTA only) and TMEM owner, warps 4..11 =
 // softmax / correction / epilogue (thread = one row x 64 keys of S, one row x 128 dims
 // of O), warp 12 = Q loader.
-// Every mbarrier wait is bounded; a
-// timeout sets MLA_DEVICE_ERR_TIMEOUT, raises a CTA-wide abort flag and the kernel
-// drains and returns.
+// Every mbarrier wait is bounded; a timeout sets MLA_DEVICE_ERR_TIMEOUT and raises a
+// CTA-wide abort flag; every role then stops issuing at its next wait (decisions that
+// several warps share go through one barrier, so they leave together), the pair drains
+// its asynchronous work and the kernel returns.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -39,11 +40,10 @@ using namespace ptx;
 
 namespace {
 
-constexpr int kNumThreads = 448;
-constexpr int kNumProducers = 4;  // warps 0, 2, 3, 13
+constexpr int kNumThreads = 384;  // 12 warps: 3 per SM sub-partition, 168 registers per thread
+constexpr int kNumProducers = 3;  // warps 0, 2, 3 (warp 0 also loads Q)
 constexpr int kMmaWarp = 1;
 constexpr int kSoftmaxWarp0 = 4;   // warps 4..11
-constexpr int kQWarp = 12;
 constexpr int kNumSoftmaxThreads = 256;
 constexpr int kStages = 7;
 constexpr int kStageBytes = 16384;
@@ -60,6 +60,8 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only whe
 constexpr uint32_t kIdescQK = make_idesc_bf16(128, 256, false, false);
 constexpr uint32_t kIdescPV = make_idesc_bf16(128, 256, false, true);
 constexpr int kBarSoftmax = 1;  // named barrier id for the 256 softmax threads
+constexpr uint64_t kDrainWaitNs = 100000000ull;  // bound on the post-abort wait for tensor-core work
+constexpr uint64_t kQuiesceNs = 500000ull;       // post-abort wait for TMA loads in flight
 
 struct Params {
   CUtensorMap tm_kv;   // [num_blocks][64][576] bf16, box {64, 64, 1}, SW128
@@ -70,6 +72,7 @@ struct Params {
   CUtensorMap tm_part;  // partial outputs as [slots][M][512] fp32, box {32, 64, 1}, SW128
   const int32_t* block_table;
   const int32_t* seqlens;
+  const int32_t* q_lens;  // per-sequence query tokens (<= s_q), or null: s_q for every sequence
   const int32_t* meta;
   __nv_bfloat16* out;
   float* lse;
@@ -82,6 +85,7 @@ struct Params {
   int B, s_q, H, M;
   float scale_log2;
   int causal;
+  int inject_stall;  // test hook: the MMA warp first waits on a barrier nothing completes
 };
 
 struct __align__(8) Ctrl {
@@ -93,8 +97,11 @@ struct __align__(8) Ctrl {
   uint64_t p_full;          // leader: P written in both CTAs (count 2)
   uint64_t p_free;          // both: PV done (commit)
   uint64_t o_free;          // leader: O read out by both CTAs (count 2)
+  uint64_t drain;           // both: every tensor-core op issued before an abort completed (commit)
+  uint64_t never;           // nothing arrives: the injected stall of the failure-path test waits on it
   uint32_t tmem_base;
   volatile int abort;
+  volatile int peer_abort;  // written by the peer CTA at teardown
   float red_max[2][4][64];
   float red_sum[4][64];   // sum of the bf16-rounded weights (normalises the output)
   float red_sum32[4][64]; // sum of the fp32 weights (gives the lse)
@@ -104,7 +111,7 @@ struct __align__(8) Ctrl {
 constexpr int kIdRing = 128;
 
 struct Piece {
-  int b, k_lo, k_hi, split, n;
+  int b, k_lo, k_hi, split, n, qlen;
 };
 
 // Block count of a sequence of n keys, or -1 when n is not a valid length for the table.
@@ -113,18 +120,28 @@ __device__ __forceinline__ int expected_blocks(const Params& p, int n) {
   return (n + kBlockSize - 1) / kBlockSize;
 }
 
+// Query tokens of sequence b: q_lens[b] when given (must lie in [0, s_q]; -1 marks an
+// invalid count), else s_q.
+__device__ __forceinline__ int query_len(const Params& p, int b) {
+  if (!p.q_lens) return p.s_q;
+  const int l = p.q_lens[b];
+  return (l < 0 || l > p.s_q) ? -1 : l;
+}
+
 // Walks the pieces of one partition.  Pieces of sequences whose length is invalid, or
 // whose block count in the metadata is not the one their current length needs (a
 // schedule built for other lengths), are skipped consistently by every role (producer
 // warp 0 writes their NaN rows).  Piece bounds are clamped to the sequence's blocks, so
-// no block-table entry past ceil(n / 64) is ever read.
+// no block-table entry past ceil(n / 64) is ever read.  With per-sequence query counts,
+// a row tile that holds only padding tokens of a sequence (rows >= q_lens[b] * H) skips
+// that sequence too; producer warp 0 writes those rows (0 / -inf).
 struct PieceWalker {
   const Params* p;
   int cb, ck, be, ke;
   const int32_t* nblk;
   const int32_t* first_part;
-  int part;
-  __device__ PieceWalker(const Params& prm, int part_) : p(&prm), part(part_) {
+  int part, row0;
+  __device__ PieceWalker(const Params& prm, int part_, int row0_) : p(&prm), part(part_), row0(row0_) {
     const int32_t* m = prm.meta;
     cb = m[off_part_start() + 2 * part];
     ck = m[off_part_start() + 2 * part + 1];
@@ -144,11 +161,14 @@ struct PieceWalker {
       if (lo >= hi) continue;
       const int n = p->seqlens[b];
       if (expected_blocks(*p, n) != nb) continue;
+      const int ql = query_len(*p, b);
+      if (ql < 0 || row0 >= ql * p->H) continue;
       pc.b = b;
       pc.k_lo = lo;
       pc.k_hi = hi;
       pc.split = part - first_part[b];
       pc.n = n;
+      pc.qlen = ql;
       return true;
     }
     return false;
@@ -263,6 +283,25 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Named barrier that also ANDs a predicate over its threads: every thread gets the same
+// answer, so a wait that ran out in one thread makes all of them leave together
+// instead of leaving the others at the next barrier.
+__device__ __forceinline__ bool named_bar_and(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %3, 0;\n\t"
+      "bar.red.and.pred q, %1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(id), "r"(count), "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -272,8 +311,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
-__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+// acc + lo(v) + hi(v) for a packed bf16 pair, with the mixed-precision f32 += bf16 add
+__device__ __forceinline__ float add_bf16x2_to(float acc, uint32_t v) {
+  float r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t.reg .f32 t;\n\tmov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.bf16 t, lo, %2;\n\tadd.rn.f32.bf16 %0, hi, t;\n\t}"
+      : "=f"(r)
+      : "r"(v), "f"(acc));
+  return r;
+}
 
 __device__ __forceinline__ int clamp_block_id(const Params& p, int32_t id) {
   if (id < 0 || (int64_t)id >= p.num_blocks) {
@@ -283,19 +329,21 @@ __device__ __forceinline__ int clamp_block_id(const Params& p, int32_t id) {
   return id;
 }
 
-// Rows of sequences that no partition covers: no visible key (out 0, lse -inf), an
-// invalid length (NaN and MLA_DEVICE_ERR_SEQLEN) or a block count in the metadata that
-// does not match the current length (NaN and MLA_DEVICE_ERR_METADATA).  Partition `part`
-// takes the sequences b with b % P == part; the 32 lanes of one warp write this CTA's
-// 64 rows [y0, y0 + 64).
-__device__ __forceinline__ void write_orphan_rows(const Params& p, int part, int P, int y0, int lane) {
+// Rows that no piece of this row tile covers: no visible key (out 0, lse -inf), a row
+// tile holding only padding tokens (0 / -inf), an invalid length or query count (NaN and
+// MLA_DEVICE_ERR_SEQLEN) or a block count in the metadata that does not match the
+// current length (NaN and MLA_DEVICE_ERR_METADATA).  Partition `part` takes the
+// sequences b with b % P == part; the 32 lanes of one warp write this CTA's 64 rows
+// [y0, y0 + 64) of the row tile that starts at row0.
+__device__ __forceinline__ void write_orphan_rows(const Params& p, int part, int P, int row0, int y0, int lane) {
   const int32_t* nblk = p.meta + off_nblk();
   for (int b = part; b < p.B; b += P) {
     const int n = p.seqlens[b];
     const int want = expected_blocks(p, n);
-    const bool bad_len = want < 0;
+    const int ql = query_len(p, b);
+    const bool bad_len = want < 0 || ql < 0;
     const bool stale = !bad_len && nblk[b] != want;
-    if (!bad_len && !stale && n > 0) continue;
+    if (!bad_len && !stale && n > 0 && row0 < ql * p.H) continue;
     const bool bad = bad_len || stale;
     const float v = bad ? __int_as_float(0x7fc00000) : 0.0f;
     const uint32_t pv = pack_bf16x2(v, v);
@@ -350,7 +398,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     mbar_init(smem_u32(&ctrl.p_full), 2);
     mbar_init(smem_u32(&ctrl.p_free), 1);
     mbar_init(smem_u32(&ctrl.o_free), 2);
+    mbar_init(smem_u32(&ctrl.drain), 1);
+    mbar_init(smem_u32(&ctrl.never), 1);
     ctrl.abort = 0;
+    ctrl.peer_abort = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -376,14 +427,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
 
   if (tile < T) {
     // =======================================================================
-    // producers: warps 0, 2, 3 and 13 own ring stages k % 4 == 0, 1, 2, 3 (one
-    // issuing warp sustains only ~half the L2 -> SM bandwidth a CTA needs; several
-    // warps issuing alternate stages of the same ring lift that limit).
+    // producers: warps 0, 2, 3 own ring stages k % 3 == 0, 1, 2 (one issuing warp
+    // sustains only about half the L2 -> SM bandwidth a CTA needs; several warps
+    // issuing alternate stages of the same ring lift that limit).  Warp 0 also loads
+    // each piece's Q.
     // =======================================================================
-    if (warp == 0 || warp == 2 || warp == 3 || warp == 13) {
-      const int pi = (warp == 0) ? 0 : (warp == 13 ? 3 : warp - 1);
+    if (warp == 0 || warp == 2 || warp == 3) {
+      const int pi = (warp == 0) ? 0 : warp - 1;
       int32_t* idwin = ctrl.block_ids[pi];
-      PieceWalker walk(p, part);
+      PieceWalker walk(p, part, tile_row0);
       uint32_t it = 0;
       bool ok = true;
       auto mine = [&]() { return (int)(it % kNumProducers) == pi; };
@@ -397,7 +449,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
       // Physical block ids of the current piece, fetched 32 at a time (one coalesced
       // load per lane) one chunk ahead of use into this warp's 128-entry window, from
       // window offset `cur_base` on; invalid ids are clamped to block 0 here (the
-      // epilogue turns that piece's rows into NaN).
+      // epilogue turns that piece's rows into NaN).  The previous piece's ids stay in
+      // the window until its last PV stages have been issued.
       Piece cur{};
       int cur_base = 0, id_pending = 0, id_chunks = 0;
       const int32_t* bt = nullptr;
@@ -472,11 +525,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           }
         }
       };
-      // Ring order per piece: QK(0), then QK(t) followed by PV(t - 1), then PV(last).
-      // The next piece is looked up one piece ahead and its first 32 block ids are
-      // loaded during the current piece's last tile, so a piece starts without
-      // waiting on the block table.
-      Piece nxt{};
+      // Q of a piece: the whole warp waits until the previous piece's last QK has
+      // completed (its Q buffer is free), then lanes 0..8 each issue one 64-column box.
+      const uint32_t q_full_l = mapa_shared(smem_u32(&ctrl.q_full), 0);
+      auto load_q = [&](const Piece& pc, int piece_idx) {
+        if (piece_idx > 0)
+          ok = __shfl_sync(0xffffffffu, wait_bar(&ctrl, p, smem_u32(&ctrl.q_empty), (piece_idx - 1) & 1, false), 0);
+        if (!ok) return;
+        const int row_base = pc.b * p.M + tile_row0 + kRowsPerCta * (int)rank;
+        expect_tx_if(lane == 0 && leader, smem_u32(&ctrl.q_full), 2 * kQBytes);
+        __syncwarp();
+        const int c = lane < kQChunks ? lane : 0;
+        tma_load_2d_cg2_if(lane < kQChunks, sQ + c * kChunkBytes, c < 8 ? (const void*)&p.tm_qn : (const void*)&p.tm_qp,
+                           q_full_l, c < 8 ? 64 * c : 0, row_base);
+      };
+      // One ring order for the whole partition: the tiles of all its pieces form one
+      // sequence, and each tile's QK stages are followed by the PV stages of the tile
+      // before it, across piece boundaries too; the last PV ends the ring.  The next
+      // piece is looked up one piece ahead and its first 32 block ids are loaded
+      // during the current piece's last tile.
+      Piece nxt{}, prv{};
+      int prv_base = 0, prv_t = -1, npieces = 0;
       bool have = walk.next(cur);
       bool have_nxt = have && walk.next(nxt);
       if (have) {
@@ -492,11 +561,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
             const int32_t* btn = p.block_table + (int64_t)nxt.b * p.max_blocks;
             id_next = (lane < nxt.k_hi - nxt.k_lo) ? clamp_block_id(p, btn[nxt.k_lo + lane]) : 0;
           }
-          issue_qk(t);
-          if (t >= 1 && ok) issue_pv(cur, cur_base, t - 1);
+          if (t == 0 && pi == 0) load_q(cur, npieces);
+          if (ok) issue_qk(t);
+          if (ok && prv_t >= 0) issue_pv(prv, prv_base, prv_t);
+          prv = cur;
+          prv_base = cur_base;
+          prv_t = t;
         }
-        if (ok) issue_pv(cur, cur_base, nt - 1);
         cur_base = (cur_base + 32 * id_chunks) % kIdRing;
+        ++npieces;
         have = have_nxt;
         if (have) {
           cur = nxt;
@@ -505,38 +578,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           have_nxt = walk.next(nxt);
         }
       }
+      if (ok && prv_t >= 0) issue_pv(prv, prv_base, prv_t);
       // With its loads issued, producer warp 0 writes the rows that no partition
       // covers while the last tiles are still being computed.
-      if (pi == 0) write_orphan_rows(p, part, P, tile_row0 + kRowsPerCta * (int)rank, lane);
-    }
-    // =======================================================================
-    // Q loader (both CTAs): Q of piece k + 1 is loaded as soon as the last QK of
-    // piece k has completed, while the MMAs still work through the PV of piece k.
-    // =======================================================================
-    else if (warp == kQWarp) {
-      // the whole warp waits (converged); lanes 0..8 each issue one 64-column box
-      PieceWalker walk(p, part);
-      Piece pc;
-      int npieces = 0;
-      const uint32_t q_full_l = mapa_shared(smem_u32(&ctrl.q_full), 0);
-      while (walk.next(pc)) {
-        if (npieces > 0 &&
-            !__shfl_sync(0xffffffffu, wait_bar(&ctrl, p, smem_u32(&ctrl.q_empty), (npieces - 1) & 1, false), 0))
-          break;
-        const int row_base = pc.b * p.M + tile_row0 + kRowsPerCta * (int)rank;
-        expect_tx_if(lane == 0 && leader, smem_u32(&ctrl.q_full), 2 * kQBytes);
-        __syncwarp();
-        const int c = lane < kQChunks ? lane : 0;
-        tma_load_2d_cg2_if(lane < kQChunks, sQ + c * kChunkBytes, c < 8 ? (const void*)&p.tm_qn : (const void*)&p.tm_qp,
-                           q_full_l, c < 8 ? 64 * c : 0, row_base);
-        ++npieces;
-      }
+      if (pi == 0) write_orphan_rows(p, part, P, tile_row0, tile_row0 + kRowsPerCta * (int)rank, lane);
     }
     // =======================================================================
     // MMA issuer (leader CTA only)
     // =======================================================================
     else if (warp == kMmaWarp && leader) {
-      PieceWalker walk(p, part);
+      // Every lane waits and the elected lane's predicate issues.  No full-warp
+      // collective sits inside the loop, so lanes that leave it at different points
+      // after a wait ran out cannot deadlock the warp; they meet again at teardown.
+      PieceWalker walk(p, part, tile_row0);
       uint32_t slot = 0, phase = 0, qk_count = 0, pv_count = 0;
       int npieces = 0;
       bool ok = true;
@@ -562,7 +616,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         for (int c = 0; c < kQChunks && ok; ++c) {
           ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), phase, false);
           if (!ok) break;
-          tc_fence_after();
           const uint64_t a0 = dq0 + c * kChunkD, b0 = dk0 + slot * kStageD;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) umma_2sm_if(elected, d, a0 + 2 * ks, b0 + 2 * ks, kIdescQK, (c | ks) != 0);
@@ -587,7 +640,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           for (int kb = 0; kb < nb && ok; ++kb) {
             ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), phase, false);
             if (!ok) break;
-            tc_fence_after();
             // the sequence's last block sits in rows [64 - rv, 64): skip whole zero steps
             const int rv = rows_in_block(pc, t, kb);
             const int ks0 = (kBlockSize - rv) >> 4;
@@ -604,19 +656,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         if (ok) commit_2sm_if(elected, smem_u32(&ctrl.p_free));
         ++pv_count;
       };
-      // same ring order as the producers
-      Piece cur;
+      // same ring order as the producers: QK of each tile, then PV of the tile before
+      Piece cur, prv{};
+      int prv_t = -1, prv_idx = 0;
+      if (p.inject_stall) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.never), 0, false);
       while (ok && walk.next(cur)) {
         ok = wait_bar(&ctrl, p, smem_u32(&ctrl.q_full), npieces & 1, false);
-        tc_fence_after();
         const int nt = num_tiles(cur);
         for (int t = 0; t < nt && ok; ++t) {
           mma_qk(nt, t);
-          if (t >= 1) mma_pv(cur, npieces, t - 1);
+          if (prv_t >= 0) mma_pv(prv, prv_idx, prv_t);
+          prv = cur;
+          prv_t = t;
+          prv_idx = npieces;
         }
-        mma_pv(cur, npieces, nt - 1);
         ++npieces;
       }
+      if (prv_t >= 0) mma_pv(prv, prv_idx, prv_t);
     }
     // =======================================================================
     // softmax / correction / epilogue
@@ -632,23 +688,106 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
       const int grow = tile_row0 + kRowsPerCta * (int)rank + m;  // row within the sequence
       const bool row_valid = grow < p.M;
       const int token = row_valid ? grow / p.H : 0;
+      const int y0 = tile_row0 + kRowsPerCta * (int)rank;
       const uint32_t p_full_l = mapa_shared(smem_u32(&ctrl.p_full), 0);
       const uint32_t o_free_l = mapa_shared(smem_u32(&ctrl.o_free), 0);
-      PieceWalker walk(p, part);
+      PieceWalker walk(p, part, tile_row0);
       Piece pc;
       uint32_t qk_count = 0, pv_count = 0;
-      bool ok = true;
-      while (ok && walk.next(pc)) {
+      // ok: this thread's waits all completed.  go: the same for all 256 threads,
+      // refreshed only by named barriers that AND ok, so every loop decision is
+      // uniform and no thread leaves the others waiting at a barrier.
+      bool ok = true, go = true;
+      // Epilogue of a finished piece: it runs once the piece's last PV has completed,
+      // inside the next piece's first tile (after that tile's weights are computed),
+      // or after the last tile.  out = O / l (bf16) or the normalised fp32 partial,
+      // written through TMA stores staged in the P buffer, which is free between a
+      // PV and the next P; then O's TMEM is handed back to the MMAs (o_free).
+      bool pend = false, pend_direct = true;
+      int pend_b = 0, pend_slot = 0;
+      float pend_sc = 0.f, pend_lse = 0.f;
+      auto epilogue = [&]() {
+        const uint32_t to = tmem + kTmemO + 128 * g + lane_off;
+        // per round every thread writes 128 bytes of its row (64 bf16 or 32 fp32 columns)
+        // into box 2g + hk, laid out [64 rows][128 B] with the 128-byte swizzle, and one
+        // thread stores the four boxes; rows past M are clipped by the tensor map
+        const uint32_t srow = sP + (2 * g + hk) * kChunkBytes + m * 128;
+        const int rounds = pend_direct ? 2 : 4;
+#pragma unroll 1
+        for (int r = 0; r < rounds; ++r) {
+          uint32_t w[32];
+          if (pend_direct) {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              uint32_t o[32];
+              tmem_ld32(to + 64 * r + 32 * hf, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int k = 0; k < 16; ++k)
+                w[16 * hf + k] =
+                    pack_bf16x2(__uint_as_float(o[2 * k]) * pend_sc, __uint_as_float(o[2 * k + 1]) * pend_sc);
+            }
+          } else {
+            tmem_ld32(to + 32 * r, w);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * pend_sc);
+          }
+          if (r > 0) named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);  // previous round's boxes were read
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(srow + ((q ^ (m & 7)) << 4)),
+                         "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
+                         : "memory");
+          fence_proxy_async_smem();
+          if (r == 0) {
+            go = named_bar_and(kBarSoftmax, kNumSoftmaxThreads, ok);
+            if (!go) return;
+          } else {
+            named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
+          }
+          if (st == 0 && y0 < p.M) {  // a CTA whose 64 rows all lie past M stores nothing
+#pragma unroll
+            for (int bx = 0; bx < 4; ++bx) {
+              const int gg = bx >> 1, hh = bx & 1;
+              if (pend_direct)
+                tma_store_3d(&p.tm_out, sP + bx * kChunkBytes, 256 * gg + 128 * hh + 64 * r, y0, pend_b);
+              else
+                tma_store_3d(&p.tm_part, sP + bx * kChunkBytes, 256 * gg + 128 * hh + 32 * r, y0, pend_slot);
+            }
+            bulk_commit();
+            bulk_wait_read_all();
+          }
+        }
+        if (row_valid && hk == 0 && g == 0) {
+          if (pend_direct)
+            p.lse[(int64_t)pend_b * p.M + grow] = pend_lse;
+          else
+            p.part_lse[(int64_t)pend_slot * p.M + grow] = pend_lse;
+        }
+        // every O read and the staging reads of the last round are done
+        tc_fence_before();
+        named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
+        if (st == 0) {
+          if (leader)
+            mbar_arrive(smem_u32(&ctrl.o_free));
+          else
+            mbar_arrive_remote(o_free_l);
+        }
+        pend = false;
+      };
+      while (go && walk.next(pc)) {
         const int nt = num_tiles(pc);
         const int piece_end = min(pc.n, pc.k_hi * kBlockSize);
-        int lim = p.causal ? (pc.n - p.s_q + token) : (pc.n - 1);
+        int lim = p.causal ? (pc.n - pc.qlen + token) : (pc.n - 1);
+        if (token >= pc.qlen) lim = -1;  // padding token: no visible key (out 0, lse -inf)
         lim = min(lim, piece_end - 1);
         if (!row_valid) lim = -1;
         // l_part: sum of the bf16 weights that enter the PV MMA (output normaliser, so
         // the weights sum to one exactly); l32_part: fp32 weights (the lse).
         float m_used = -INFINITY, l_part = 0.f, l32_part = 0.f;
         // Block-id validity and split layout of the piece (loads issued now, consumed
-        // at the epilogue).
+        // at the piece's end).
         const int nsplit = p.meta[off_num_splits(p.B) + pc.b];
         const int split_base = p.meta[off_split_prefix(p.B) + pc.b];
         int bad_ids = 0;
@@ -659,10 +798,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
             bad_ids |= (id < 0 || (int64_t)id >= p.num_blocks);
           }
         }
-        for (int t = 0; t < nt && ok; ++t) {
+        for (int t = 0; t < nt && go; ++t) {
           const uint32_t buf = qk_count & 1;
-          ok = wait_bar(&ctrl, p, smem_u32(&ctrl.s_full[buf]), (qk_count >> 1) & 1, false);
-          if (!ok) break;
+          // A wait that runs out does not leave the loop here: the thread carries on to
+          // the next AND barrier, which makes all 256 threads leave together.
+          ok = wait_bar(&ctrl, p, smem_u32(&ctrl.s_full[buf]), (qk_count >> 1) & 1, false) && ok;
           tc_fence_after();
           uint32_t sr[64];
           {
@@ -676,15 +816,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           const int key0 = (pc.k_lo + t * kBlocksPerTile) * kBlockSize + 128 * hk + 64 * g;
           int cnt = lim - key0 + 1;
           cnt = cnt < 0 ? 0 : (cnt > 64 ? 64 : cnt);
-          float lmax = -INFINITY;
+          // Tiles with every key visible (all but a sequence's last tile and causal
+          // edges) take an unmasked path; the choice is warp-uniform.
+          const bool full = __all_sync(0xffffffffu, cnt == kBlockSize);
+          // Row maximum of the raw scores (the scale is positive, so it keeps their
+          // order), over four independent chains.
+          float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+          if (full) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float x = __uint_as_float(sr[c]) * p.scale_log2;
-            sr[c] = __float_as_uint(x);
-            if (c < cnt) lmax = fmaxf(lmax, x);
+            for (int c = 0; c < 64; c += 4) {
+              mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
+              mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+              mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
+              mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; c += 4) {
+              if (c < cnt) mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
+              if (c + 1 < cnt) mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+              if (c + 2 < cnt) mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
+              if (c + 3 < cnt) mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
+            }
           }
+          const float lmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
           ctrl.red_max[qk_count & 1][2 * hk + g][m] = lmax;
-          named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
+          go = named_bar_and(kBarSoftmax, kNumSoftmaxThreads, ok);
+          if (!go) break;
           float rmax = ctrl.red_max[qk_count & 1][0][m];
           rmax = fmaxf(rmax, ctrl.red_max[qk_count & 1][1][m]);
           rmax = fmaxf(rmax, ctrl.red_max[qk_count & 1][2][m]);
@@ -698,27 +856,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
             l_part *= alpha;
             l32_part *= alpha;
           }
-          const float mref = (m_used == -INFINITY) ? 0.f : m_used;
+          const float nref = (m_used == -INFINITY) ? 0.f : -m_used;
+          const float sl2 = p.scale_log2;
           uint32_t pk[32];
-          float lsum = 0.f, lsum32 = 0.f;
+          // weights 2^(s * scale_log2 - m); sums of the bf16-rounded weights (output
+          // normaliser) and of the fp32 weights (lse), two chains each
+          float ls0 = 0.f, ls1 = 0.f, lf0 = 0.f, lf1 = 0.f;
+          if (full) {
 #pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            const float e0 = (c < cnt) ? fast_exp2(__uint_as_float(sr[c]) - mref) : 0.f;
-            const float e1 = (c + 1 < cnt) ? fast_exp2(__uint_as_float(sr[c + 1]) - mref) : 0.f;
-            const uint32_t v = pack_bf16x2(e0, e1);
-            pk[c >> 1] = v;
-            lsum += bf16lo(v) + bf16hi(v);
-            lsum32 += e0 + e1;
+            for (int c = 0; c < 64; c += 4) {
+              const float e0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, nref));
+              const float e1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, nref));
+              const float e2 = fast_exp2(fmaf(__uint_as_float(sr[c + 2]), sl2, nref));
+              const float e3 = fast_exp2(fmaf(__uint_as_float(sr[c + 3]), sl2, nref));
+              const uint32_t v0 = pack_bf16x2(e0, e1), v1 = pack_bf16x2(e2, e3);
+              pk[c >> 1] = v0;
+              pk[(c >> 1) + 1] = v1;
+              ls0 = add_bf16x2_to(ls0, v0);
+              ls1 = add_bf16x2_to(ls1, v1);
+              lf0 += e0 + e1;
+              lf1 += e2 + e3;
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; c += 4) {
+              const float e0 = (c < cnt) ? fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, nref)) : 0.f;
+              const float e1 = (c + 1 < cnt) ? fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, nref)) : 0.f;
+              const float e2 = (c + 2 < cnt) ? fast_exp2(fmaf(__uint_as_float(sr[c + 2]), sl2, nref)) : 0.f;
+              const float e3 = (c + 3 < cnt) ? fast_exp2(fmaf(__uint_as_float(sr[c + 3]), sl2, nref)) : 0.f;
+              const uint32_t v0 = pack_bf16x2(e0, e1), v1 = pack_bf16x2(e2, e3);
+              pk[c >> 1] = v0;
+              pk[(c >> 1) + 1] = v1;
+              ls0 = add_bf16x2_to(ls0, v0);
+              ls1 = add_bf16x2_to(ls1, v1);
+              lf0 += e0 + e1;
+              lf1 += e2 + e3;
+            }
           }
-          l_part += lsum;
-          l32_part += lsum32;
-          // PV of the previous tile must be done before P is overwritten / O rescaled.
-          if (t >= 1) {
-            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1, false);
-            if (!ok) break;
+          l_part += ls0 + ls1;
+          l32_part += lf0 + lf1;
+          // PV of the previous tile (possibly the previous piece's last) must be done
+          // before P is overwritten, O is rescaled or the previous piece's O is read.
+          if (qk_count >= 1) {
+            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1, false) && ok;
             ++pv_count;
             tc_fence_after();
-            if (__any_sync(0xffffffffu, rescale)) {
+            if (t == 0) {
+              if (pend) {
+                epilogue();
+                if (!go) break;
+              }
+            } else if (__any_sync(0xffffffffu, rescale)) {
               const uint32_t to = tmem + kTmemO + 128 * g + lane_off;
 #pragma unroll 1
               for (int c = 0; c < 128; c += 32) {
@@ -786,10 +974,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           }
           ++qk_count;
         }
-        if (!ok) break;
-        // ---- epilogue of the piece ----------------------------------------
-        // Row sums and the block-id verdict are final after the last tile's P: reduce
-        // them while the last PV is still running.
+        if (!go) break;
+        // ---- end of the piece: row sums and the block-id verdict are final; reduce
+        // them while its last PV is still running, and keep what its epilogue needs
         ctrl.red_sum[2 * hk + g][m] = l_part;
         ctrl.red_sum32[2 * hk + g][m] = l32_part;
         if (st == 0) ctrl.bad_piece = 0;
@@ -800,82 +987,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
             ctrl.red_sum32[0][m] + ctrl.red_sum32[1][m] + ctrl.red_sum32[2][m] + ctrl.red_sum32[3][m];
         named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
         const bool bad = ctrl.bad_piece != 0;
-        const bool direct = (nsplit == 1);
         const float nanf_ = __int_as_float(0x7fc00000);
-        const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
-        const float lse_val =
-            bad ? nanf_ : ((l32_row > 0.f) ? (m_used + __log2f(l32_row)) * 0.69314718055994531f : -INFINITY);
-        const int64_t orow = (int64_t)pc.b * p.M + grow;
-        const int64_t slot = (int64_t)split_base + pc.split;
-        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1, false);
-        if (!ok) break;
+        // a bad piece's rows become NaN: scaling by NaN turns every value into NaN
+        pend_sc = bad ? nanf_ : ((l_row > 0.f) ? 1.f / l_row : 0.f);
+        pend_lse = bad ? nanf_ : ((l32_row > 0.f) ? (m_used + __log2f(l32_row)) * 0.69314718055994531f : -INFINITY);
+        pend_direct = (nsplit == 1);
+        pend_b = pc.b;
+        pend_slot = split_base + pc.split;
+        pend = true;
+      }
+      // the last piece's epilogue, after its last PV (the AND makes the decision uniform)
+      go = named_bar_and(kBarSoftmax, kNumSoftmaxThreads, ok && go);
+      if (go && pend) {
+        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1, false) && ok;
         ++pv_count;
         tc_fence_after();
-        const uint32_t to = tmem + kTmemO + 128 * g + lane_off;
-        // a bad piece's rows become NaN: scaling by NaN turns every value into NaN
-        const float sc = bad ? nanf_ : inv_l;
-        // The output leaves through TMA stores staged in the P buffer (unused until the
-        // next piece's first P): per round every thread writes 128 bytes of its row
-        // (64 bf16 or 32 fp32 columns) into box 2g + hk, laid out [64 rows][128 B] with
-        // the 128-byte swizzle, and one thread stores the four boxes.  Rows past M are
-        // clipped by the tensor map.
-        const uint32_t srow = sP + (2 * g + hk) * kChunkBytes + m * 128;
-        const int rounds = direct ? 2 : 4;
-        const int y0 = tile_row0 + kRowsPerCta * (int)rank;
-#pragma unroll 1
-        for (int r = 0; r < rounds; ++r) {
-          uint32_t w[32];
-          if (direct) {
-            uint32_t o0[32], o1[32];
-            tmem_ld32(to + 64 * r, o0);
-            tmem_ld32(to + 64 * r + 32, o1);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              w[k] = pack_bf16x2(__uint_as_float(o0[2 * k]) * sc, __uint_as_float(o0[2 * k + 1]) * sc);
-              w[16 + k] = pack_bf16x2(__uint_as_float(o1[2 * k]) * sc, __uint_as_float(o1[2 * k + 1]) * sc);
-            }
-          } else {
-            tmem_ld32(to + 32 * r, w);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * sc);
-          }
-          if (r > 0) named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);  // previous round's boxes were read
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(srow + ((q ^ (m & 7)) << 4)),
-                         "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
-                         : "memory");
-          fence_proxy_async_smem();
-          named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
-          if (st == 0 && y0 < p.M) {  // a CTA whose 64 rows all lie past M stores nothing
-#pragma unroll
-            for (int bx = 0; bx < 4; ++bx) {
-              const int gg = bx >> 1, hh = bx & 1;
-              if (direct)
-                tma_store_3d(&p.tm_out, sP + bx * kChunkBytes, 256 * gg + 128 * hh + 64 * r, y0, pc.b);
-              else
-                tma_store_3d(&p.tm_part, sP + bx * kChunkBytes, 256 * gg + 128 * hh + 32 * r, y0, (int)slot);
-            }
-            bulk_commit();
-            bulk_wait_read_all();
-          }
-        }
-        if (row_valid && hk == 0 && g == 0) {
-          if (direct)
-            p.lse[orow] = lse_val;
-          else
-            p.part_lse[slot * p.M + grow] = lse_val;
-        }
-        tc_fence_before();
-        named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
-        if (st == 0) {
-          if (leader)
-            mbar_arrive(smem_u32(&ctrl.o_free));
-          else
-            mbar_arrive_remote(o_free_l);
-        }
+        epilogue();
       }
     }
   }
@@ -884,8 +1011,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
   if (warp == kSoftmaxWarp0 && lane == 0) bulk_wait_all();  // the epilogue's TMA stores landed
   tc_fence_before();
   __syncthreads();
-  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  // Every role has stopped issuing (all waits are bounded).  Each CTA tells the other
+  // whether it aborted; then both drain together or neither does.
+  if (tid == 0) st_cluster_u32(mapa_shared(smem_u32((const void*)&ctrl.peer_abort), rank ^ 1u), (uint32_t)ctrl.abort);
+  cluster_sync();
   tc_fence_after();
+  if (ctrl.abort || ctrl.peer_abort) {
+    // A wait ran out somewhere in the pair: asynchronous work issued before it may still
+    // be in flight.  Tensor-core work (MMAs) has a completion handle: a commit issued
+    // after it arrives on both CTAs' drain barriers once all of it has completed.  TMA
+    // loads have none besides the stage barriers that did not complete, so both CTAs
+    // also wait out their latency (at most a few microseconds even under full load)
+    // with a 500 us margin before the TMEM and the shared memory are released.
+    if (warp == kMmaWarp) {
+      const bool el = elect_one();
+      if (leader) commit_2sm_if(el, smem_u32(&ctrl.drain));
+      const uint64_t dl = globaltimer_ns() + kDrainWaitNs;
+      while (!mbar_try_wait(smem_u32(&ctrl.drain), 0) && globaltimer_ns() < dl) {
+      }
+    }
+    if (tid == 0) {
+      const uint64_t until = globaltimer_ns() + kQuiesceNs;
+      while (globaltimer_ns() < until) {
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    tc_fence_after();
+  }
   if (warp == kMmaWarp) {
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
@@ -906,9 +1060,10 @@ cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
                           const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
                           const CUtensorMap& tm_out, const CUtensorMap& tm_part,
                           const int32_t* block_table, int max_blocks, const int32_t* seqlens,
-                          const int32_t* meta, int64_t num_blocks, int B, int s_q, int H, float scale,
-                          int causal, void* out, float* lse, float* part_o, float* part_lse,
-                          int32_t* status, int num_ctas, cudaStream_t stream) {
+                          const int32_t* q_lens, const int32_t* meta, int64_t num_blocks, int B, int s_q,
+                          int H, float scale, int causal, void* out, float* lse, float* part_o, float* part_lse,
+                          int32_t* status, int num_ctas, uint64_t wait_timeout_ns, int inject_stall,
+                          cudaStream_t stream) {
   Params prm;
   prm.tm_kv = tm_kv;
   prm.tm_kv2 = tm_kv2;
@@ -918,6 +1073,7 @@ cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
   prm.tm_part = tm_part;
   prm.block_table = block_table;
   prm.seqlens = seqlens;
+  prm.q_lens = q_lens;
   prm.meta = meta;
   prm.out = reinterpret_cast<__nv_bfloat16*>(out);
   prm.lse = lse;
@@ -925,7 +1081,7 @@ cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
   prm.part_lse = part_lse;
   prm.status = status;
   prm.num_blocks = num_blocks;
-  prm.timeout_ns = 1000000000ull;
+  prm.timeout_ns = wait_timeout_ns;
   prm.max_blocks = max_blocks;
   prm.B = B;
   prm.s_q = s_q;
@@ -933,6 +1089,7 @@ cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
   prm.M = s_q * H;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.causal = causal;
+  prm.inject_stall = inject_stall;
   mla_decode_kernel<<<num_ctas, kNumThreads, kSmemDyn + 1024, stream>>>(prm);
   return cudaGetLastError();
 }

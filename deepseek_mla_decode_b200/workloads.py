@@ -161,3 +161,17 @@ def make_inputs(
 def make_workload(name: str, **kw) -> DecodeInputs:
     w = WORKLOADS[name]
     return make_inputs(w.B, w.s_q, w.H, w.seqlens(), w.seed, causal=w.causal, **kw)
+
+
+def make_up_projections(H: int, seed: int, scale: float = 0.05):
+    """Per-head up-projection weights W_UK, W_UV [H, 128, 512] as bf16 bit patterns,
+    drawn N(0, scale^2) (random stand-ins for trained weights)."""
+    rng = np.random.default_rng(seed)
+    w_uk = f32_to_bf16_bits(rng.standard_normal((H, 128, D_LATENT), dtype=np.float32) * np.float32(scale))
+    w_uv = f32_to_bf16_bits(rng.standard_normal((H, 128, D_LATENT), dtype=np.float32) * np.float32(scale))
+    return w_uk, w_uv
+
+
+def make_rows(shape, seed: int):
+    """bf16 bit patterns of N(0, 1) draws with the given shape."""
+    return _normal_bf16(np.random.default_rng(seed), shape)

@@ -59,7 +59,8 @@ typedef enum {
 
 /* Bits OR-ed into the optional device status word by the kernels. */
 #define MLA_DEVICE_ERR_BLOCK_ID 1 /* block_table entry outside [0, num_blocks) */
-#define MLA_DEVICE_ERR_SEQLEN 2   /* cache_seqlens[b] < 0 or > max_blocks * 64  */
+#define MLA_DEVICE_ERR_SEQLEN 2   /* cache_seqlens[b] < 0 or > max_blocks * 64,
+                                     or q_lens[b] outside [0, s_q]               */
 #define MLA_DEVICE_ERR_TIMEOUT 4  /* an internal bounded wait ran out           */
 #define MLA_DEVICE_ERR_METADATA 8 /* metadata not produced for these B, s_q, H, or
                                      for another length of some sequence (its block
@@ -139,6 +140,28 @@ mla_status_t mla_decode(const void* q_nope, const void* q_pe, const void* kv_cac
                         void* out, float* lse, int32_t* status, void* stream);
 
 /*
+ * mla_decode with a per-sequence number of query tokens: sequence b has
+ * q_lens[b] <= s_q new tokens (speculative decoding where sequences accept different
+ * numbers of draft tokens -- Paddle 3.0 inference upgrade article, speculative
+ * decoding section).  Its tokens are the last q_lens[b] cache positions: with causal
+ * != 0, token i sees keys 0 .. n_b - q_lens[b] + i.  Tokens i >= q_lens[b] are padding:
+ * their out rows are 0 and their lse -inf.  q and out keep the padded
+ * [B, s_q, H, ...] layout.
+ *
+ *   q_lens  device int32 [B], each in [0, s_q]; NULL means s_q for every sequence
+ *           (then the call is mla_decode).  A value outside [0, s_q] makes that
+ *           sequence's rows NaN and sets MLA_DEVICE_ERR_SEQLEN.
+ * Other arguments, the metadata and the workspace are those of mla_decode.  A 128-row
+ * tile of query rows that holds only padding tokens of a sequence is not computed.
+ */
+mla_status_t mla_decode_ragged(const void* q_nope, const void* q_pe, const void* kv_cache,
+                               int64_t num_blocks, const int32_t* block_table, int max_blocks,
+                               const int32_t* cache_seqlens, const int32_t* q_lens, int B, int s_q,
+                               int H, float softmax_scale, int causal, const void* metadata,
+                               size_t metadata_bytes, void* workspace, size_t workspace_bytes,
+                               void* out, float* lse, int32_t* status, void* stream);
+
+/*
  * The two launches mla_decode performs, exposed separately (same arguments, same
  * semantics; mla_decode == mla_decode_attention followed by mla_decode_combine on
  * the same stream with the same workspace).
@@ -195,6 +218,47 @@ mla_status_t mla_decode_noalloc(const void* q_nope, const void* q_pe, const void
                                 float softmax_scale, int causal, const void* metadata,
                                 size_t metadata_bytes, void* out, float* lse, int32_t* status,
                                 void* stream);
+
+/*
+ * Failure-path test hooks, process-wide, for launches made after the call.  Library
+ * conveniences: no passage of the source pages corresponds to them, and production
+ * code never needs them.
+ *
+ * mla_set_wait_timeout_ns: bound on every internal mbarrier wait of the attention
+ *   kernel, in nanoseconds (ns = 0 restores the default of 1 s).  A wait that runs
+ *   out sets MLA_DEVICE_ERR_TIMEOUT: every role of the kernel stops issuing work, the
+ *   CTA pair waits for the tensor-core work and the TMA loads it had in flight, and
+ *   the kernel returns with that call's outputs undefined.
+ * mla_set_stall_injection: nonzero makes the attention kernel's MMA warp first wait
+ *   on a barrier that nothing ever completes, so that wait and then the others run
+ *   out -- the way the timeout path is exercised without a faulty kernel.  0 turns
+ *   it off.
+ */
+mla_status_t mla_set_wait_timeout_ns(uint64_t ns);
+mla_status_t mla_set_stall_injection(int enable);
+
+/*
+ * Weight-absorption GEMMs either side of the decode (KsanaLLM 0.6.0 release notes,
+ * section 2.1, WA-MLA).  With per-head up-projections k_h = W_UK[h] c and
+ * v_h = W_UV[h] c of the 512-d latent c, and query rows r = b * s_q + i (R rows):
+ *
+ * mla_absorb_q:   q_nope[r, h, :] = W_UK[h]^T q_heads[r, h, :]
+ *   q_heads  bf16 [R, H, 128]   per-head no-RoPE queries
+ *   w_uk     bf16 [H, 128, 512] key up-projections (row k of W_UK[h] is 512 wide)
+ *   q_nope   bf16 [R, H, 512]   written: the absorbed query mla_decode takes
+ * mla_absorb_out: y[r, h, :] = W_UV[h] o[r, h, :]
+ *   o_latent bf16 [R, H, 512]   the decode output
+ *   w_uv     bf16 [H, 128, 512] value up-projections
+ *   y        bf16 [R, H, 128]   written: per-head attention output
+ *
+ * fp32 accumulation, bf16 results (round to nearest even).  Pointers are device
+ * pointers, 16-byte aligned; 1 <= R, 1 <= H <= 65535.  Asynchronous on `stream`;
+ * host-detectable errors return before any launch.
+ */
+mla_status_t mla_absorb_q(const void* q_heads, const void* w_uk, void* q_nope, int R, int H,
+                          void* stream);
+mla_status_t mla_absorb_out(const void* o_latent, const void* w_uv, void* y, int R, int H,
+                            void* stream);
 
 /* Number of streaming multiprocessors the schedule targets on the current device.
  * Library convenience: no passage of the source pages corresponds to it. */

@@ -42,12 +42,14 @@ def run_cuda(inp, dev=None, status=None):
     return out.float().cpu().double().numpy(), lse.cpu().double().numpy(), meta
 
 
-def oracle(inp, seqs=None):
-    """Oracle outputs, optionally for a subset of sequences only."""
+def oracle(inp, seqs=None, q_lens=None):
+    """Oracle outputs, optionally for a subset of sequences only, optionally with
+    per-sequence query counts."""
     qn, qp = O.bf16_to_f64(inp.q_nope), O.bf16_to_f64(inp.q_pe)
     kv = O.bf16_to_f64(inp.kv_cache) if seqs is None else None
     if seqs is None:
-        return O.mla_decode_ref(qn, qp, kv, inp.block_table, inp.cache_seqlens, inp.softmax_scale, inp.causal)
+        return O.mla_decode_ref(qn, qp, kv, inp.block_table, inp.cache_seqlens, inp.softmax_scale, inp.causal,
+                                q_lens=q_lens)
     outs, lses = [], []
     for b in seqs:
         n = int(inp.cache_seqlens[b])
@@ -56,7 +58,8 @@ def oracle(inp, seqs=None):
         kv_b = O.bf16_to_f64(inp.kv_cache[ids])  # only this sequence's blocks
         table = np.arange(max(nblk, 1))[None, :]
         o, l = O.mla_decode_ref(qn[b : b + 1], qp[b : b + 1], kv_b if nblk else np.zeros((1, 64, 576)), table,
-                                np.array([n]), inp.softmax_scale, inp.causal)
+                                np.array([n]), inp.softmax_scale, inp.causal,
+                                q_lens=None if q_lens is None else np.asarray(q_lens)[b : b + 1])
         outs.append(o[0])
         lses.append(l[0])
     return np.stack(outs), np.stack(lses)

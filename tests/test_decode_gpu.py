@@ -52,6 +52,42 @@ def test_more_draft_tokens(s_q):
     check(make_inputs(2, s_q, 128, [129, 1030], seed=50 + s_q, causal=True))
 
 
+@pytest.mark.parametrize("H,s_q,q_lens,lens", [
+    (64, 4, [4, 1, 2, 0, 3], [300, 1000, 77, 500, 2000]),   # two row tiles: tokens {0,1} and {2,3}
+    (128, 2, [1, 2, 0, 1, 2], [5000, 129, 64, 9000, 1]),    # one row tile per token; long splits
+    (16, 3, [3, 2, 1], [1, 2, 700]),                        # fewer keys than query tokens
+])
+def test_ragged_query_counts(H, s_q, q_lens, lens):
+    inp = make_inputs(len(lens), s_q, H, lens, seed=80 + H + s_q, causal=True)
+    dev = to_device(inp)
+    ql = torch.tensor(q_lens, dtype=torch.int32, device="cuda")
+    meta = mla.get_metadata(dev["cache_seqlens"], s_q, H)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = mla.decode_ragged(dev["q_nope"], dev["q_pe"], dev["kv_cache"], dev["block_table"],
+                                 dev["cache_seqlens"], ql, inp.softmax_scale, True, meta, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_out, ref_lse = oracle(inp, q_lens=np.array(q_lens))
+    compare(out.float().cpu().double().numpy(), lse.cpu().double().numpy(), ref_out, ref_lse,
+            what=f"ragged H={H} s_q={s_q}")
+
+
+def test_ragged_invalid_query_count():
+    inp = make_inputs(3, 2, 64, [100, 300, 50], seed=90, causal=True)
+    dev = to_device(inp)
+    ql = torch.tensor([2, 3, 1], dtype=torch.int32, device="cuda")  # 3 > s_q
+    meta = mla.get_metadata(dev["cache_seqlens"], 2, 64)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = mla.decode_ragged(dev["q_nope"], dev["q_pe"], dev["kv_cache"], dev["block_table"],
+                                 dev["cache_seqlens"], ql, inp.softmax_scale, True, meta, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == mla.MLA_DEVICE_ERR_SEQLEN
+    out, lse = out.float().cpu().double().numpy(), lse.cpu().double().numpy()
+    assert np.all(np.isnan(out[1])) and np.all(np.isnan(lse[1]))
+    ref_out, ref_lse = oracle(inp, [0, 2], q_lens=np.array([2, 2, 1]))
+    compare(out[[0, 2]], lse[[0, 2]], ref_out, ref_lse)
+
+
 def test_single_long_sequence_split():
     # one sequence long enough to be cut into many pieces + LSE combine
     check(make_inputs(1, 1, 128, [20000], seed=61))
@@ -189,6 +225,28 @@ def test_metadata_for_other_lengths():
     good = [0, 2, 3]
     ref_out, ref_lse = oracle(inp, good)
     compare(out[good], lse[good], ref_out, ref_lse)
+
+
+def test_wait_timeout_sets_status_and_returns():
+    """The MMA warp waits on a barrier nothing completes (a test hook), bounded by
+    1 ms: the kernel must set the timeout bit, stop every role, drain what the pair
+    had in flight and return, leaving the context usable -- the next call, with the
+    default bound, is exact."""
+    inp = make_inputs(3, 1, 128, [3000, 700, 5000], seed=71)
+    dev = to_device(inp)
+    meta = mla.get_metadata(dev["cache_seqlens"], 1, 128)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    try:
+        mla.set_wait_timeout_ns(1_000_000)
+        mla.set_stall_injection(True)
+        mla.decode(dev["q_nope"], dev["q_pe"], dev["kv_cache"], dev["block_table"], dev["cache_seqlens"],
+                   inp.softmax_scale, False, meta, status=status)
+        torch.cuda.synchronize()
+    finally:
+        mla.set_stall_injection(False)
+        mla.set_wait_timeout_ns(0)
+    assert int(status.item()) & mla.MLA_DEVICE_ERR_TIMEOUT
+    check(inp)
 
 
 def test_host_argument_errors():
