@@ -39,6 +39,7 @@ EXPORTED_SYMBOLS = (
     "mla_set_stall_injection",
     "mla_absorb_q",
     "mla_absorb_out",
+    "mla_quantize_kv_fp8",
 )
 
 _lib = None
@@ -89,6 +90,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for fn in (L.mla_absorb_q, L.mla_absorb_out):
         fn.restype = c_int
         fn.argtypes = [c_vp, c_vp, c_vp, c_int, c_int, c_vp]
+    L.mla_quantize_kv_fp8.restype = c_int
+    L.mla_quantize_kv_fp8.argtypes = [c_vp, c_vp, c_i64, c_vp]
     L.mla_decode_noalloc.restype = c_int
     L.mla_decode_noalloc.argtypes = [c_vp, c_vp, c_vp, c_i64, c_vp, c_int, c_vp, c_int, c_int, c_int, c_f, c_int,
                                      c_vp, c_size, c_vp, c_vp, c_vp, c_vp]
@@ -243,6 +246,21 @@ def absorb_out(o_latent, w_uv, y=None, stream=None):
     _check("mla_absorb_out", load_library().mla_absorb_out(o_latent.data_ptr(), w_uv.data_ptr(), y.data_ptr(), R, H,
                                                            _stream_ptr(stream)))
     return y
+
+
+def quantize_kv_fp8(kv_cache, kv_fp8=None, stream=None):
+    """mla_quantize_kv_fp8: bf16 cache [num_blocks, 64, 576] -> packed FP8 rows
+    [num_blocks, 64, 656] (uint8)."""
+    import torch
+
+    if kv_cache.shape[-1] != 576 or not kv_cache.is_contiguous():
+        raise ValueError("contiguous [..., 576] bf16 cache expected")
+    rows = kv_cache.numel() // 576
+    if kv_fp8 is None:
+        kv_fp8 = torch.empty((*kv_cache.shape[:-1], 656), dtype=torch.uint8, device=kv_cache.device)
+    _check("mla_quantize_kv_fp8", load_library().mla_quantize_kv_fp8(kv_cache.data_ptr(), kv_fp8.data_ptr(), rows,
+                                                                     _stream_ptr(stream)))
+    return kv_fp8
 
 
 def decode_attention(q_nope, q_pe, kv_cache, block_table, cache_seqlens, softmax_scale: float, causal: bool,

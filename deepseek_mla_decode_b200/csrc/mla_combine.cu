@@ -33,6 +33,8 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
     const int32_t* __restrict__ meta, const int32_t* __restrict__ seqlens, const int32_t* __restrict__ q_lens,
     int max_blocks, int B, int s_q, int M, const float* __restrict__ part_o, const float* __restrict__ part_lse,
     __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  // launched as a programmatic dependent of the attention kernel: wait for it
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int part = blockIdx.x;
   if (part == 0) return;
   const int b = meta[off_part_start() + 2 * part];
@@ -98,10 +100,18 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
 cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, const int32_t* q_lens, int max_blocks,
                            int B, int s_q, int M, int P, const float* part_o, const float* part_lse, void* out, float* lse,
                            cudaStream_t stream) {
-  dim3 grid(P, (M + kWarps - 1) / kWarps);
-  combine_kernel<<<grid, kWarps * 32, 0, stream>>>(meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o, part_lse,
-                                                   reinterpret_cast<__nv_bfloat16*>(out), lse);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P, (M + kWarps - 1) / kWarps);
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o, part_lse,
+                            reinterpret_cast<__nv_bfloat16*>(out), lse);
 }
 
 }  // namespace mla

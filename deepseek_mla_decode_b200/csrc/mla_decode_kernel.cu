@@ -374,18 +374,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = (rank == 0);
   const int worker = blockIdx.x >> 1;
-  const int P = p.meta[kHdrNumParts];
-  int T = p.meta[kHdrNumTiles];
-  if (p.meta[kHdrMagic] != kMetaMagic || p.meta[kHdrB] != p.B || p.meta[kHdrSq] != p.s_q ||
-      p.meta[kHdrH] != p.H || P * T * 2 != (int)gridDim.x) {
-    if (tid == 0 && blockIdx.x == 0) set_status(p, kErrMetadata);
-    T = 0;  // every role skips; the CTA still joins the cluster barriers below
-  }
-  const int tile = worker / P;
-  const int part = worker % P;
-  const int tile_row0 = tile * kRowsPerTile;
 
-  // ---- setup ---------------------------------------------------------------
+  // ---- setup (reads no input: it overlaps the previous kernel's tail when this one
+  // is launched as a programmatic dependent) -----------------------------------
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&ctrl.full[s]), 1);
@@ -424,6 +415,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
   tc_fence_after();
   const uint32_t tmem = ctrl.tmem_base;
+  // Inputs may come from the previous kernel in the stream (the schedule): wait for
+  // it to complete, then let the next kernel (the LSE combine) start launching.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int P = p.meta[kHdrNumParts];
+  int T = p.meta[kHdrNumTiles];
+  if (p.meta[kHdrMagic] != kMetaMagic || p.meta[kHdrB] != p.B || p.meta[kHdrSq] != p.s_q ||
+      p.meta[kHdrH] != p.H || P * T * 2 != (int)gridDim.x) {
+    if (tid == 0 && blockIdx.x == 0) set_status(p, kErrMetadata);
+    T = 0;  // every role skips; the CTA still joins the cluster barriers below
+  }
+  const int tile = worker / P;
+  const int part = worker % P;
+  const int tile_row0 = tile * kRowsPerTile;
 
   if (tile < T) {
     // =======================================================================
@@ -1090,8 +1095,20 @@ cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.causal = causal;
   prm.inject_stall = inject_stall;
-  mla_decode_kernel<<<num_ctas, kNumThreads, kSmemDyn + 1024, stream>>>(prm);
-  return cudaGetLastError();
+  // Programmatic dependent launch: the CTAs start (and run their setup) while the
+  // previous kernel in the stream finishes; the kernel waits for it before reading
+  // any input.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_ctas);
+  cfg.blockDim = dim3(kNumThreads);
+  cfg.dynamicSmemBytes = kSmemDyn + 1024;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mla_decode_kernel, prm);
 }
 
 }  // namespace mla

@@ -18,10 +18,9 @@ namespace mla {
 
 namespace {
 
-constexpr int kThreads = 1024;
-
 // Block-wide exclusive scan of int64 values held one per thread; returns the
 // exclusive prefix for this thread and writes the block total to *total.
+template <int kThreads>
 __device__ int64_t block_exclusive_scan(int64_t v, int64_t* scratch /*[32]*/, int64_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int64_t x = v;
@@ -48,11 +47,17 @@ __device__ int64_t block_exclusive_scan(int64_t v, int64_t* scratch /*[32]*/, in
   return warp_excl + x - v;
 }
 
+// kThreads = 256 for batches of at most 256 sequences (fewer and cheaper block-wide
+// barriers), 1024 otherwise.
+template <int kThreads>
 __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __restrict__ seqlens, int B,
                                                             int s_q, int H, int num_workers,
                                                             int32_t* __restrict__ meta) {
   __shared__ int64_t scratch[32];
   __shared__ int64_t s_carry, s_total;
+  // the attention kernel that follows may start its setup now (it waits for this
+  // kernel to complete before reading the schedule)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int tid = threadIdx.x;
   const int M = s_q * H;
   const int T = (M + kRowsPerTile - 1) / kRowsPerTile;
@@ -76,7 +81,7 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
     const int64_t nt = (nb + kBlocksPerTile - 1) / kBlocksPerTile;
     const int64_t cost = nb > 0 ? nt + kSchedOverheadTiles : 0;
     int64_t total;
-    const int64_t pre = block_exclusive_scan(cost, scratch, &total);
+    const int64_t pre = block_exclusive_scan<kThreads>(cost, scratch, &total);
     int64_t cap = (total + P - 1) / P;
     if (cap < kSchedMinCap) cap = kSchedMinCap;
     for (int q = tid; q < kMaxWorkers; q += kThreads) {
@@ -106,7 +111,7 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
       num_splits[b] = (int32_t)ns;
     }
     int64_t total_slots;
-    const int64_t ex = block_exclusive_scan(ns, scratch, &total_slots);
+    const int64_t ex = block_exclusive_scan<kThreads>(ns, scratch, &total_slots);
     if (b < B) split_prefix[b] = (int32_t)ex;
     __syncthreads();
     for (int q = tid; q < kMaxWorkers; q += kThreads) {
@@ -146,7 +151,7 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
       cost = nb > 0 ? (nb + kBlocksPerTile - 1) / kBlocksPerTile + kSchedOverheadTiles : 0;
     }
     int64_t t;
-    block_exclusive_scan(cost, scratch, &t);
+    block_exclusive_scan<kThreads>(cost, scratch, &t);
     total += t;
   }
   int64_t cap = (total + P - 1) / P;
@@ -171,7 +176,7 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
       cost = nb > 0 ? (nb + kBlocksPerTile - 1) / kBlocksPerTile + kSchedOverheadTiles : 0;
     }
     int64_t chunk_total;
-    const int64_t pre = s_carry + block_exclusive_scan(cost, scratch, &chunk_total);
+    const int64_t pre = s_carry + block_exclusive_scan<kThreads>(cost, scratch, &chunk_total);
     if (b < B) {
       if (nb > 0) {
         const int64_t first_pos = pre + kSchedOverheadTiles;
@@ -205,7 +210,7 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
     const int b = base + tid;
     const int64_t v = (b < B) ? num_splits[b] : 0;
     int64_t chunk_total;
-    const int64_t ex = s_carry + block_exclusive_scan(v, scratch, &chunk_total);
+    const int64_t ex = s_carry + block_exclusive_scan<kThreads>(v, scratch, &chunk_total);
     if (b < B) split_prefix[b] = (int32_t)ex;
     __syncthreads();
     if (tid == 0) s_carry += chunk_total;
@@ -243,7 +248,10 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
 
 cudaError_t launch_metadata(const int32_t* seqlens, int B, int s_q, int H, int num_workers,
                             int32_t* meta, cudaStream_t stream) {
-  metadata_kernel<<<1, kThreads, 0, stream>>>(seqlens, B, s_q, H, num_workers, meta);
+  if (B <= 256)
+    metadata_kernel<256><<<1, 256, 0, stream>>>(seqlens, B, s_q, H, num_workers, meta);
+  else
+    metadata_kernel<1024><<<1, 1024, 0, stream>>>(seqlens, B, s_q, H, num_workers, meta);
   return cudaGetLastError();
 }
 

@@ -260,6 +260,22 @@ mla_status_t mla_absorb_q(const void* q_heads, const void* w_uk, void* q_nope, i
 mla_status_t mla_absorb_out(const void* o_latent, const void* w_uv, void* y, int R, int H,
                             void* stream);
 
+/*
+ * FP8 (e4m3) latent cache.  8-bit KV-cache inference is among the serving
+ * capabilities of the Paddle 3.0 inference upgrade article (closing list); the
+ * per-token max-abs scale follows the quantised KV cache of the "DeepSeek speed test"
+ * article, section 3.1.  The packed row (656 bytes, this library's format):
+ *   [0, 512)    e4m3 codes of c_kv (OCP E4M3FN)   [512, 640)  k_pe, 64 bf16
+ *   [640, 644)  fp32 scale = max|c_kv| / 448      [644, 656)  zero
+ * with code = e4m3(c / scale): IEEE fp32 quotient, rounded to nearest even, saturated
+ * to +-448; a zero row has scale 0 and zero codes.  Dequantised c = scale * e4m3(code).
+ *
+ * mla_quantize_kv_fp8: quantise `rows` bf16 cache rows [rows, 576] into packed rows
+ *   [rows, 656] (for a paged cache, rows = num_blocks * 64).  Device pointers, 16-byte
+ *   aligned; asynchronous on `stream`.
+ */
+mla_status_t mla_quantize_kv_fp8(const void* kv_cache, void* kv_fp8, int64_t rows, void* stream);
+
 /* Number of streaming multiprocessors the schedule targets on the current device.
  * Library convenience: no passage of the source pages corresponds to it. */
 mla_status_t mla_device_sm_count(int* sm_count);
