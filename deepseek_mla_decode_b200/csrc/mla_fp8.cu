@@ -5,16 +5,20 @@
 // inference upgrade article (closing capabilities list); scaling each token's cached
 // vector by its own max-abs value follows the per-token quantised KV cache of the
 // "DeepSeek speed test" article, section 3.1.  The row format is this library's own:
-//     bytes [0, 512)    e4m3 codes of c_kv            (OCP E4M3FN, no infinities)
-//     bytes [512, 640)  k_pe, 64 bf16, unchanged       (RoPE keys keep 16 bits)
-//     bytes [640, 644)  fp32 scale = max|c_kv| / 448   (448 = largest finite e4m3)
+//     bytes [0, 512)    e4m3 codes of c_kv / scale     (OCP E4M3FN, no infinities)
+//     bytes [512, 640)  k_pe / scale as 64 bf16         (RoPE keys keep 16 bits)
+//     bytes [640, 644)  fp32 scale = max|row| / 448     (over all 576 values;
+//                                                        448 = largest finite e4m3)
 //     bytes [644, 656)  zero
-// and code_i = e4m3(c_i / scale): the quotient is an IEEE fp32 division, rounded to
-// the nearest e4m3 value (ties to even) and saturated to +-448; a row whose c_kv is
-// all zero gets scale 0 and zero codes.  The dequantised latent is scale * e4m3(code).
+// code_i = e4m3(c_i / scale): the quotient is an IEEE fp32 division, rounded to the
+// nearest e4m3 value (ties to even) and saturated to +-448; k_pe'_j = bf16(k_pe_j /
+// scale), the fp32 quotient rounded to nearest even.  A row of zeros gets scale 0 and
+// stores zeros.  The dequantised row is scale * [e4m3(code) | k_pe'], so one scale
+// multiplies the whole score q . k and the whole value row.
 //
-// One warp per cache row: lane l holds c_kv[16 l, 16 l + 16), a warp max gives the
-// scale, and each lane writes its 16 codes as one 16-byte store.
+// One warp per cache row: lane l holds c_kv[16 l, 16 l + 16) and lanes 0-7 also hold
+// k_pe[8 l, 8 l + 8); a warp max gives the scale, and each lane writes its 16 codes
+// (and its 8 scaled k_pe values) as 16-byte stores.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -51,13 +55,27 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) quantize_kernel(const __n
     c[2 * i] = __uint_as_float(w[i] << 16);
     c[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
   }
+  // k_pe[8 lane .. 8 lane + 7] on lanes 0-7
+  float k[8];
+  {
+    const uint4 e = lane < 8 ? reinterpret_cast<const uint4*>(src + kDLatent)[lane] : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t v[4] = {e.x, e.y, e.z, e.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      k[2 * i] = __uint_as_float(v[i] << 16);
+      k[2 * i + 1] = __uint_as_float(v[i] & 0xffff0000u);
+    }
+  }
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(c[i]));
 #pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(k[i]));
+#pragma unroll
   for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   const float scale = __fdiv_rn(amax, 448.0f);
   uint32_t q[4] = {0u, 0u, 0u, 0u};
+  uint32_t kq[4] = {0u, 0u, 0u, 0u};
   if (scale > 0.f) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -65,11 +83,16 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) quantize_kernel(const __n
       const uint32_t hi = e4m3x2(__fdiv_rn(c[4 * i + 2], scale), __fdiv_rn(c[4 * i + 3], scale));
       q[i] = lo | (hi << 16);
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(__fdiv_rn(k[2 * i], scale), __fdiv_rn(k[2 * i + 1], scale));
+      kq[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
   }
   reinterpret_cast<uint4*>(dst)[lane] = make_uint4(q[0], q[1], q[2], q[3]);
-  // k_pe (128 bytes) by lanes 0-7, then the scale and the zero pad by lane 8
+  // scaled k_pe (128 bytes) by lanes 0-7, then the scale and the zero pad by lane 8
   if (lane < 8) {
-    reinterpret_cast<uint4*>(dst + 512)[lane] = reinterpret_cast<const uint4*>(src + kDLatent)[lane];
+    reinterpret_cast<uint4*>(dst + 512)[lane] = make_uint4(kq[0], kq[1], kq[2], kq[3]);
   } else if (lane == 8) {
     reinterpret_cast<uint4*>(dst + 640)[0] = make_uint4(__float_as_uint(scale), 0u, 0u, 0u);
   }

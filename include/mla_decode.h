@@ -265,10 +265,13 @@ mla_status_t mla_absorb_out(const void* o_latent, const void* w_uv, void* y, int
  * capabilities of the Paddle 3.0 inference upgrade article (closing list); the
  * per-token max-abs scale follows the quantised KV cache of the "DeepSeek speed test"
  * article, section 3.1.  The packed row (656 bytes, this library's format):
- *   [0, 512)    e4m3 codes of c_kv (OCP E4M3FN)   [512, 640)  k_pe, 64 bf16
- *   [640, 644)  fp32 scale = max|c_kv| / 448      [644, 656)  zero
+ *   [0, 512)    e4m3 codes of c_kv / scale (OCP E4M3FN)
+ *   [512, 640)  k_pe / scale as 64 bf16
+ *   [640, 644)  fp32 scale = max|row| / 448 over all 576 values
+ *   [644, 656)  zero
  * with code = e4m3(c / scale): IEEE fp32 quotient, rounded to nearest even, saturated
- * to +-448; a zero row has scale 0 and zero codes.  Dequantised c = scale * e4m3(code).
+ * to +-448, and k_pe' = bf16(k_pe / scale) rounded to nearest even; a zero row has
+ * scale 0 and stores zeros.  The dequantised row is scale * [e4m3(code) | k_pe'].
  *
  * mla_quantize_kv_fp8: quantise `rows` bf16 cache rows [rows, 576] into packed rows
  *   [rows, 656] (for a paged cache, rows = num_blocks * 64).  Device pointers, 16-byte

@@ -15,21 +15,25 @@ Sources (page titles and sections):
 The pages give no FP8 cache format.  The readings taken here (each is listed in
 DESIGN.md):
 
-1. Only the 512-wide latent ``c_kv`` is quantised; the 64-wide RoPE key ``k_pe``
-   stays bf16 (it is 11 % of the row and carries position information).
-2. One fp32 scale per token (per cache row): ``scale = amax / 448`` with
-   ``amax = max |c_kv|`` and 448 the largest finite e4m3 value; both computed in
-   fp32.  The code of value ``c`` is ``e4m3(c / scale)``: the fp32 quotient (IEEE
-   division, round to nearest even) rounded to e4m3 to nearest even, saturating
-   to +-448.  A row with ``amax = 0`` has scale 0 and all codes 0.
+1. One fp32 scale per token (per cache row) for the whole 576-wide row:
+   ``scale = amax / 448`` with ``amax = max |row|`` over c_kv and k_pe, and 448 the
+   largest finite e4m3 value; both computed in fp32.
+2. The 512-wide latent ``c_kv`` is quantised: the code of value ``c`` is
+   ``e4m3(c / scale)``, the fp32 quotient (IEEE division, round to nearest even)
+   rounded to e4m3 to nearest even, saturating to +-448.  The 64-wide RoPE key
+   ``k_pe`` keeps 16 bits (it is 11 % of the row and carries position
+   information) and is stored in the same scaled units: ``bf16(k_pe / scale)``,
+   the fp32 quotient rounded to bf16 to nearest even.  A row with ``amax = 0`` has
+   scale 0 and stores zeros.  Every stored row is then ``scale * [codes | k_pe']``.
 3. e4m3 is the OCP "E4M3FN" encoding: 1 sign, 4 exponent (bias 7), 3 mantissa
    bits, no infinities, NaN = S.1111.111, largest finite 448, smallest subnormal
    2^-9.  The sign of zero is kept (-0 encodes as 0x80).
 4. A cache row is packed into 656 bytes: bytes [0, 512) the e4m3 codes of c_kv,
-   [512, 640) k_pe as 64 bf16, [640, 644) the fp32 scale, [644, 656) zero.
-5. The dequantised latent is ``scale * e4m3_value(code)`` (exact in float64), and
-   decode over the FP8 cache is the bf16 definition (``mla_oracle.mla_decode_ref``)
-   applied to the dequantised rows.
+   [512, 640) the scaled k_pe as 64 bf16, [640, 644) the fp32 scale, [644, 656)
+   zero.
+5. The dequantised row is ``scale * [e4m3_value(codes) | k_pe']`` (exact in
+   float64), and decode over the FP8 cache is the bf16 definition
+   (``mla_oracle.mla_decode_ref``) applied to the dequantised rows.
 
 Parity: the decode table, the encoder and the quantiser are pinned in
 ``tests/test_fp8_oracle_pins.py`` by hand-checked codes, round trips, tie and
@@ -94,19 +98,27 @@ def e4m3_encode(x: np.ndarray) -> np.ndarray:
     return (sign | mag.astype(np.uint8)).astype(np.uint8)
 
 
-def quantize_rows(c_kv_bf16: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
-    """Per-token quantisation of bf16 latent rows [..., 512] (uint16 bit patterns).
+def f32_to_bf16_rne(x: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bit patterns, round to nearest even (finite inputs)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    return ((u + (np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1)))) >> np.uint32(16)).astype(np.uint16)
 
-    Returns (codes uint8 [..., 512], scale float32 [...]): scale = amax / 448 and
-    code = e4m3(c / scale), every step in float32 as stated above."""
-    c = O.bf16_to_f64(c_kv_bf16).astype(np.float32)  # exact
-    amax = np.max(np.abs(c), axis=-1)  # float32, exact
+
+def quantize_rows(rows_bf16: np.ndarray) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Per-token quantisation of bf16 cache rows [..., 576] (uint16 bit patterns).
+
+    Returns (codes uint8 [..., 512], k_pe' uint16 [..., 64], scale float32 [...]):
+    scale = amax / 448 over the whole row, codes = e4m3(c / scale) and
+    k_pe' = bf16(k_pe / scale), every step in float32 as stated above."""
+    r = O.bf16_to_f64(rows_bf16).astype(np.float32)  # exact
+    amax = np.max(np.abs(r), axis=-1)  # float32, exact
     scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)  # IEEE fp32 division
     safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
-    q = (c / safe[..., None]).astype(np.float32)  # IEEE fp32 division
-    codes = e4m3_encode(q)
-    codes = np.where((scale > 0)[..., None], codes, np.uint8(0)).astype(np.uint8)
-    return codes, scale
+    q = (r / safe[..., None]).astype(np.float32)  # IEEE fp32 division
+    live = (scale > 0)[..., None]
+    codes = np.where(live, e4m3_encode(q[..., : O.D_LATENT]), np.uint8(0)).astype(np.uint8)
+    kpe = np.where(live, f32_to_bf16_rne(q[..., O.D_LATENT :]), np.uint16(0)).astype(np.uint16)
+    return codes, kpe, scale
 
 
 def pack_cache(kv_cache_bf16: np.ndarray) -> np.ndarray:
@@ -114,17 +126,17 @@ def pack_cache(kv_cache_bf16: np.ndarray) -> np.ndarray:
     [num_blocks, 64, 656] (uint8) in the row format stated above."""
     nb, bs, d = kv_cache_bf16.shape
     assert bs == O.BLOCK_SIZE and d == O.D_QK
-    codes, scale = quantize_rows(kv_cache_bf16[..., : O.D_LATENT])
+    codes, kpe, scale = quantize_rows(kv_cache_bf16)
     out = np.zeros((nb, bs, ROW_BYTES), dtype=np.uint8)
     out[..., :OFF_KPE] = codes
-    kpe = np.ascontiguousarray(kv_cache_bf16[..., O.D_LATENT :], dtype=np.uint16)
-    out[..., OFF_KPE:OFF_SCALE] = kpe.view(np.uint8).reshape(nb, bs, 2 * O.D_ROPE)
+    out[..., OFF_KPE:OFF_SCALE] = np.ascontiguousarray(kpe).view(np.uint8).reshape(nb, bs, 2 * O.D_ROPE)
     out[..., OFF_SCALE : OFF_SCALE + 4] = np.ascontiguousarray(scale, dtype=np.float32).view(np.uint8).reshape(nb, bs, 4)
     return out
 
 
 def unpack_cache(packed: np.ndarray) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
-    """Packed FP8 cache -> (codes uint8 [..., 512], k_pe uint16 [..., 64], scale float32 [...])."""
+    """Packed FP8 cache -> (codes uint8 [..., 512], scaled k_pe uint16 [..., 64],
+    scale float32 [...])."""
     packed = np.ascontiguousarray(packed, dtype=np.uint8)
     codes = packed[..., :OFF_KPE]
     kpe = np.ascontiguousarray(packed[..., OFF_KPE:OFF_SCALE]).view(np.uint16)
@@ -133,10 +145,10 @@ def unpack_cache(packed: np.ndarray) -> Tuple[np.ndarray, np.ndarray, np.ndarray
 
 
 def dequantize_cache(packed: np.ndarray) -> np.ndarray:
-    """Packed FP8 cache -> float64 rows [..., 576] = [scale * e4m3(codes) | k_pe]."""
+    """Packed FP8 cache -> float64 rows [..., 576] = scale * [e4m3(codes) | k_pe']."""
     codes, kpe, scale = unpack_cache(packed)
-    c = e4m3_decode(codes) * scale.astype(np.float64)[..., None]
-    return np.concatenate([c, O.bf16_to_f64(kpe)], axis=-1)
+    s = scale.astype(np.float64)[..., None]
+    return np.concatenate([e4m3_decode(codes) * s, O.bf16_to_f64(kpe) * s], axis=-1)
 
 
 def mla_decode_fp8_ref(q_nope, q_pe, kv_fp8_packed, block_table, cache_seqlens, softmax_scale, causal):

@@ -53,11 +53,17 @@ def test_ties_go_to_even_code_and_saturation():
 
 def test_quantiser_error_bound_and_scale():
     inp = make_inputs(2, 1, 16, [300, 200], seed=5)
-    rows = inp.kv_cache[..., :512]
-    codes, scale = F.quantize_rows(rows)
-    c = O.bf16_to_f64(rows)
-    amax = np.max(np.abs(c), axis=-1)
+    rows = inp.kv_cache
+    codes, kpe, scale = F.quantize_rows(rows)
+    r = O.bf16_to_f64(rows)
+    amax = np.max(np.abs(r), axis=-1)
     assert np.array_equal(scale, (amax.astype(np.float32) / np.float32(448.0)).astype(np.float32))
+    # k_pe' = k_pe / scale to within half a bf16 ulp (2^-8 relative: 8 significant
+    # bits) plus the fp32 quotient's rounding
+    kq = r[..., 512:] / scale[..., None].astype(np.float64)
+    kd = O.bf16_to_f64(kpe)
+    assert np.all(np.abs(kd - kq) <= np.abs(kq) * (2.0 ** -8 + 2.0 ** -23) + 1e-30)
+    c = r[..., :512]
     x = c / scale[..., None].astype(np.float64)  # exact quotient
     deq = F.e4m3_decode(codes)
     a = np.abs(deq)
@@ -66,16 +72,17 @@ def test_quantiser_error_bound_and_scale():
     spacing = np.where(a < 2.0 ** -6, 2.0 ** -9, 2.0 ** (e - 3))
     # quotient rounded to fp32 first, then to e4m3: half a spacing plus the fp32 rounding
     assert np.all(np.abs(x - deq) <= spacing / 2 * (1 + 2.0 ** -20) + np.abs(x) * 2.0 ** -23)
-    # the largest element of each row maps to +-448 exactly
+    # where the row maximum lies in c_kv it maps to +-448 exactly
+    in_c = np.max(np.abs(c), axis=-1) == amax
     arg = np.argmax(np.abs(c), axis=-1)
     top = np.take_along_axis(codes, arg[..., None], axis=-1)[..., 0]
-    assert np.all((top == 0x7E) | (top == 0xFE))
+    assert in_c.any() and np.all(((top == 0x7E) | (top == 0xFE))[in_c])
 
 
 def test_zero_row_has_zero_scale_and_codes():
-    rows = np.zeros((1, 64, 512), dtype=np.uint16)
-    codes, scale = F.quantize_rows(rows)
-    assert np.all(scale == 0) and np.all(codes == 0)
+    rows = np.zeros((1, 64, 576), dtype=np.uint16)
+    codes, kpe, scale = F.quantize_rows(rows)
+    assert np.all(scale == 0) and np.all(codes == 0) and np.all(kpe == 0)
 
 
 def test_packed_row_layout():
@@ -83,17 +90,16 @@ def test_packed_row_layout():
     packed = F.pack_cache(inp.kv_cache)
     assert packed.shape == (inp.kv_cache.shape[0], 64, 656)
     codes, kpe, scale = F.unpack_cache(packed)
-    assert np.array_equal(kpe, inp.kv_cache[..., 512:])
     assert np.all(packed[..., 644:] == 0)
-    c2, s2 = F.quantize_rows(inp.kv_cache[..., :512])
-    assert np.array_equal(codes, c2) and np.array_equal(scale, s2)
+    c2, k2, s2 = F.quantize_rows(inp.kv_cache)
+    assert np.array_equal(codes, c2) and np.array_equal(kpe, k2) and np.array_equal(scale, s2)
 
 
 def test_fp8_decode_equals_bf16_decode_on_exact_rows():
-    """Rows whose latent values are e4m3 values with a 448 in each row quantise with
-    scale 1 and codes equal to the values, so the FP8 decode must equal the bf16
-    decode bit for bit."""
-    inp = make_inputs(3, 2, 16, [70, 130, 5], seed=7, causal=True)
+    """Rows whose latent values are e4m3 values with a 448 in each row (and k_pe
+    within +-448) quantise with scale 1, codes equal to the values and k_pe stored
+    unchanged, so the FP8 decode must equal the bf16 decode bit for bit."""
+    inp = make_inputs(3, 2, 16, [70, 130, 5], seed=7, causal=True, poison=False)
     rng = np.random.default_rng(8)
     grid = F.E4M3_VALUES[:127][F.E4M3_VALUES[:127] <= 8.0]
     vals = rng.choice(grid, size=inp.kv_cache[..., :512].shape) * rng.choice([-1.0, 1.0], size=inp.kv_cache[..., :512].shape)
@@ -110,10 +116,10 @@ def test_fp8_decode_equals_bf16_decode_on_exact_rows():
 
 
 def test_fp8_decode_within_perturbation_bound_of_bf16_decode():
-    """Quantisation moves each latent value by delta; a score moves by at most
-    Delta = scale * sum |q_nope| |delta| (k_pe is unchanged), so every weight changes by
-    a factor within exp(+-2 Delta) and the weights' total variation is at most
-    exp(2 Delta) - 1.  Hence |out - out8| <= max |delta| + (exp(2 Delta) - 1) max |c|
+    """Quantisation moves each stored value by delta (latent and RoPE parts); a score
+    moves by at most Delta = scale * sum |q| |delta|, so every weight changes by a
+    factor within exp(+-2 Delta) and the weights' total variation is at most
+    exp(2 Delta) - 1.  Hence |out - out8| <= max |delta_c| + (exp(2 Delta) - 1) max |c|
     per query row, and |lse - lse8| <= Delta."""
     inp = make_inputs(2, 1, 32, [500, 900], seed=9)
     packed = F.pack_cache(inp.kv_cache)
@@ -125,11 +131,12 @@ def test_fp8_decode_within_perturbation_bound_of_bf16_decode():
     orig = O.bf16_to_f64(inp.kv_cache)
     for b in range(inp.B):
         n = int(inp.cache_seqlens[b])
-        r16 = O.gather_rows(orig, inp.block_table[b], n)[:, :512]
-        r8 = O.gather_rows(deq, inp.block_table[b], n)[:, :512]
+        r16 = O.gather_rows(orig, inp.block_table[b], n)
+        r8 = O.gather_rows(deq, inp.block_table[b], n)
         delta = np.abs(r8 - r16)
-        big_delta = inp.softmax_scale * (np.abs(qn[b, 0]) @ delta.T).max(axis=-1)  # [H]
-        bound = delta.max() + (np.exp(2 * big_delta) - 1) * np.abs(r16).max()
+        q = np.concatenate([qn[b, 0], qp[b, 0]], axis=-1)
+        big_delta = inp.softmax_scale * (np.abs(q) @ delta.T).max(axis=-1)  # [H]
+        bound = delta[:, :512].max() + (np.exp(2 * big_delta) - 1) * np.abs(r16[:, :512]).max()
         err = np.abs(o8[b, 0] - o16[b, 0]).max(axis=-1)
         assert np.all(err <= bound), (err.max(), bound.min())
         assert np.all(np.abs(l8[b, 0] - l16[b, 0]) <= big_delta * (1 + 1e-12))
