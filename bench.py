@@ -44,9 +44,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # ---------------------------------------------------------------------------
 # algorithmic work (per call)
 # ---------------------------------------------------------------------------
-def algorithmic_work(seqlens, s_q, H, causal):
+def algorithmic_work(seqlens, s_q, H, causal, row_bytes=D_QK * 2):
     """FLOPs = 2 (576 + 512) per (sequence, query token, visible key, head);
-    cache bytes = every visible cache row once (1152 B per (sequence, key));
+    cache bytes = every visible cache row once (row_bytes per (sequence, key): 1152 B
+    for the bf16 cache, 656 B for the packed FP8 cache);
     algorithmic bytes = cache bytes + q + out + lse."""
     flops = 0
     keys = 0
@@ -56,7 +57,7 @@ def algorithmic_work(seqlens, s_q, H, causal):
             vis = n if not causal else max(0, min(n, n - s_q + i + 1))
             flops += max(vis, 0) * H * 2 * (D_QK + D_LATENT)
     B = len(seqlens)
-    cache_bytes = keys * D_QK * 2
+    cache_bytes = keys * row_bytes
     q_bytes = B * s_q * H * D_QK * 2
     out_bytes = B * s_q * H * D_LATENT * 2 + B * s_q * H * 4
     return flops, cache_bytes, cache_bytes + q_bytes + out_bytes
@@ -242,10 +243,10 @@ class DeviceRun:
     """One workload resident on the device, stepped through the C ABI: schedule,
     attention and LSE combine, each bracketed by CUDA events on the launching stream."""
 
-    def __init__(self, mla, inp, dev):
+    def __init__(self, mla, inp, dev, fp8=False):
         import torch
 
-        self.mla, self.inp, self.dev = mla, inp, dev
+        self.mla, self.inp, self.dev, self.fp8 = mla, inp, dev, fp8
 
         def bf16(bits):
             return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
@@ -260,6 +261,9 @@ class DeviceRun:
         self.lse = torch.empty((B, s_q, H), dtype=torch.float32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.stream = torch.cuda.current_stream()
+        if fp8:  # the packed FP8 cache, quantised once (outside every timed region)
+            self.kv = mla.quantize_kv_fp8(self.kv)
+            torch.cuda.synchronize()
 
     def _step(self, ev=None):
         m, i, st = self.mla, self.inp, self.stream
@@ -268,8 +272,12 @@ class DeviceRun:
         m.get_metadata(self.seqlens, i.s_q, i.H, metadata=self.meta, stream=st)
         if ev is not None:
             ev[1].record(st)
-        m.decode_attention(self.q_nope, self.q_pe, self.kv, self.table, self.seqlens, i.softmax_scale, i.causal,
-                           self.meta, self.ws, self.out, self.lse, status=self.status, stream=st)
+        if self.fp8:
+            m.decode_fp8_attention(self.q_nope, self.q_pe, self.kv, self.table, self.seqlens, i.softmax_scale,
+                                   i.causal, self.meta, self.ws, self.out, self.lse, status=self.status, stream=st)
+        else:
+            m.decode_attention(self.q_nope, self.q_pe, self.kv, self.table, self.seqlens, i.softmax_scale, i.causal,
+                               self.meta, self.ws, self.out, self.lse, status=self.status, stream=st)
         if ev is not None:
             ev[2].record(st)
         m.decode_combine(self.seqlens, self.table.shape[1], i.s_q, i.H, self.meta, self.ws, self.out, self.lse,
@@ -350,7 +358,7 @@ class DeviceRun:
         return e0.elapsed_time(e1) / n, h2d, d2h
 
 
-def roofline(inp, t, steps):
+def roofline(inp, t, steps, fp8=False):
     """Roofline figures of the attention kernel from summed device milliseconds.
 
     Roofline time = max(cache bytes / HBM peak, FLOPs / bf16 peak); `achieved` is the
@@ -359,7 +367,8 @@ def roofline(inp, t, steps):
     pct_of_roofline_decode the same over the whole mla_decode call (attention +
     combine)."""
     hbm_peak, tc_peak, _, peak_src = load_peaks()
-    flops, cache_bytes, algo_bytes = algorithmic_work(inp.cache_seqlens, inp.s_q, inp.H, inp.causal)
+    flops, cache_bytes, algo_bytes = algorithmic_work(inp.cache_seqlens, inp.s_q, inp.H, inp.causal,
+                                                      656 if fp8 else D_QK * 2)
     att_s = t["attention"] / steps * 1e-3
     t_hbm = cache_bytes / (hbm_peak * 1e9)
     t_tc = flops / (tc_peak * 1e12)
@@ -371,7 +380,8 @@ def roofline(inp, t, steps):
         achieved = flops / att_s / 1e12
         r = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s", "frac": achieved / tc_peak,
              "peak_source": f"{peak_src} (burst bf16 GEMM)"}
-    r["kernel"] = "mla_decode_kernel (split-KV attention)"
+    r["kernel"] = "mla_decode_kernel<fp8> (split-KV attention, FP8 cache)" if fp8 else \
+        "mla_decode_kernel (split-KV attention)"
     r["kernel_avg_us"] = att_s * 1e6
     r["roofline_us"] = max(t_hbm, t_tc) * 1e6
     r["pct_of_roofline"] = max(t_hbm, t_tc) / att_s
@@ -504,6 +514,17 @@ def main():
             torch.cuda.synchronize()
             ri.check_status(name)
             per_workload[name] = roofline(wi, ti, args.per_workload_steps)
+            del ri
+            torch.cuda.empty_cache()
+        # the four full-size decode configurations over the packed FP8 cache (656-byte rows)
+        for name in ("serving_b256", "decode_b64", "mtp_b128_sq2", "long_b4"):
+            wi = make_workload(name)
+            ri = DeviceRun(mla, wi, dev, fp8=True)
+            ri.steps(args.warmup, flusher)
+            ti = ri.steps(args.per_workload_steps, flusher, timed=True)
+            torch.cuda.synchronize()
+            ri.check_status(name + " (fp8)")
+            per_workload[name + "_fp8"] = roofline(wi, ti, args.per_workload_steps, fp8=True)
             del ri
             torch.cuda.empty_cache()
 

@@ -40,6 +40,8 @@ EXPORTED_SYMBOLS = (
     "mla_absorb_q",
     "mla_absorb_out",
     "mla_quantize_kv_fp8",
+    "mla_decode_fp8",
+    "mla_decode_fp8_attention",
 )
 
 _lib = None
@@ -85,8 +87,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for fn in (L.mla_decode, L.mla_decode_attention):
         fn.restype = c_int
         fn.argtypes = dec_args
-    L.mla_decode_ragged.restype = c_int
-    L.mla_decode_ragged.argtypes = dec_args[:7] + [c_vp] + dec_args[7:]
+    for fn in (L.mla_decode_ragged, L.mla_decode_fp8, L.mla_decode_fp8_attention):
+        fn.restype = c_int
+        fn.argtypes = dec_args[:7] + [c_vp] + dec_args[7:]
     for fn in (L.mla_absorb_q, L.mla_absorb_out):
         fn.restype = c_int
         fn.argtypes = [c_vp, c_vp, c_vp, c_int, c_int, c_vp]
@@ -210,6 +213,31 @@ def decode_ragged(q_nope, q_pe, kv_cache, block_table, cache_seqlens, q_lens, so
                         workspace, out, lse, status, stream)
     _check("mla_decode_ragged", load_library().mla_decode_ragged(*args[:7], q_lens.data_ptr(), *args[7:]))
     return out, lse
+
+
+def decode_fp8(q_nope, q_pe, kv_fp8, block_table, cache_seqlens, softmax_scale: float, causal: bool, metadata,
+               q_lens=None, workspace=None, out=None, lse=None, status=None, stream=None) -> Tuple[object, object]:
+    """mla_decode_fp8: the decode over a packed FP8 cache [num_blocks, 64, 656] (uint8,
+    as written by quantize_kv_fp8); q_lens as in decode_ragged, or None."""
+    if kv_fp8.shape[-1] != 656:
+        raise ValueError("packed FP8 cache [num_blocks, 64, 656] expected")
+    workspace, out, lse = _alloc_outputs(q_nope, workspace, out, lse)
+    if q_lens is not None and not q_lens.is_contiguous():
+        raise ValueError("q_lens must be contiguous")
+    args = _decode_args(q_nope, q_pe, kv_fp8, block_table, cache_seqlens, softmax_scale, causal, metadata,
+                        workspace, out, lse, status, stream)
+    _check("mla_decode_fp8", load_library().mla_decode_fp8(*args[:7], q_lens.data_ptr() if q_lens is not None
+                                                           else None, *args[7:]))
+    return out, lse
+
+
+def decode_fp8_attention(q_nope, q_pe, kv_fp8, block_table, cache_seqlens, softmax_scale: float, causal: bool,
+                         metadata, workspace, out, lse, q_lens=None, status=None, stream=None):
+    """The FP8 split-KV attention launch alone (see mla_decode_fp8_attention)."""
+    args = _decode_args(q_nope, q_pe, kv_fp8, block_table, cache_seqlens, softmax_scale, causal, metadata,
+                        workspace, out, lse, status, stream)
+    _check("mla_decode_fp8_attention", load_library().mla_decode_fp8_attention(
+        *args[:7], q_lens.data_ptr() if q_lens is not None else None, *args[7:]))
 
 
 def absorb_q(q_heads, w_uk, q_nope=None, stream=None):

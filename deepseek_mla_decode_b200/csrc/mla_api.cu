@@ -17,7 +17,8 @@ cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, const in
                            int B, int s_q, int M, int P, const float* part_o, const float* part_lse, void* out,
                            float* lse, cudaStream_t stream);
 cudaError_t decode_kernel_setup(int device);
-cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
+cudaError_t launch_decode(bool fp8, const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
+                          const CUtensorMap* tm_kpe, const CUtensorMap* tm_scl,
                           const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
                           const CUtensorMap& tm_out, const CUtensorMap& tm_part,
                           const int32_t* block_table, int max_blocks, const int32_t* seqlens,
@@ -101,10 +102,11 @@ int parts_for(int num_workers, int s_q, int H) {
 }
 
 bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
-            const cuuint32_t* box, CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+            const cuuint32_t* box, CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+            CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint32_t es[4] = {1, 1, 1, 1};
   return g_encode(m, dt, rank, const_cast<void*>(base), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -225,15 +227,47 @@ mla_status_t check_decode_args(const void* q_nope, const void* q_pe, const void*
   return MLA_OK;
 }
 
-mla_status_t launch_attention(const void* q_nope, const void* q_pe, const void* kv_cache, int64_t num_blocks,
-                              const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
-                              const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
-                              const void* metadata,
-                              void* workspace, void* out, float* lse, int32_t* status, const DecodeGeom& g,
-                              cudaStream_t s) {
-  const int64_t rows = static_cast<int64_t>(B) * g.M;
-  CUtensorMap tm_kv, tm_kv2, tm_qn, tm_qp;
+// FP8 cache views (rows of kRowBytes8 bytes): code slabs for QK (64 columns, no swizzle)
+// and PV (128 columns, 128-byte swizzle), the scaled k_pe as bf16 and the scales as fp32.
+bool encode_fp8_cache(const void* kv, int64_t num_blocks, CUtensorMap* tm_q, CUtensorMap* tm_v, CUtensorMap* tm_kpe,
+                      CUtensorMap* tm_scl) {
+  const cuuint64_t row = mla::kRowBytes8, blk = (cuuint64_t)mla::kRowBytes8 * mla::kBlockSize;
   {
+    cuuint64_t dims[3] = {row, (cuuint64_t)mla::kBlockSize, (cuuint64_t)num_blocks};
+    cuuint64_t strides[2] = {row, blk};
+    cuuint32_t box_q[3] = {64, 64, 1};
+    cuuint32_t box_v[3] = {128, 64, 1};
+    if (!encode(tm_q, kv, 3, dims, strides, box_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode(tm_v, kv, 3, dims, strides, box_v, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_128B))
+      return false;
+  }
+  {
+    cuuint64_t dims[3] = {row / 2, (cuuint64_t)mla::kBlockSize, (cuuint64_t)num_blocks};
+    cuuint64_t strides[2] = {row, blk};
+    cuuint32_t box[3] = {64, 64, 1};
+    if (!encode(tm_kpe, kv, 3, dims, strides, box)) return false;
+  }
+  {
+    cuuint64_t dims[3] = {row / 4, (cuuint64_t)mla::kBlockSize, (cuuint64_t)num_blocks};
+    cuuint64_t strides[2] = {row, blk};
+    cuuint32_t box[3] = {4, 64, 1};
+    if (!encode(tm_scl, kv, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  }
+  return true;
+}
+
+mla_status_t launch_attention(bool fp8, const void* q_nope, const void* q_pe, const void* kv_cache,
+                              int64_t num_blocks, const int32_t* block_table, int max_blocks,
+                              const int32_t* cache_seqlens, const int32_t* q_lens, int B, int s_q, int H,
+                              float softmax_scale, int causal, const void* metadata, void* workspace, void* out,
+                              float* lse, int32_t* status, const DecodeGeom& g, cudaStream_t s) {
+  const int64_t rows = static_cast<int64_t>(B) * g.M;
+  CUtensorMap tm_kv, tm_kv2, tm_qn, tm_qp, tm_kpe, tm_scl;
+  if (fp8) {
+    if (!encode_fp8_cache(kv_cache, num_blocks, &tm_kv, &tm_kv2, &tm_kpe, &tm_scl)) return MLA_ERR_INVALID_ARG;
+  } else {
+    {
     cuuint64_t dims[3] = {(cuuint64_t)mla::kDQK, (cuuint64_t)mla::kBlockSize, (cuuint64_t)num_blocks};
     cuuint64_t strides[2] = {(cuuint64_t)mla::kDQK * 2, (cuuint64_t)mla::kDQK * 2 * mla::kBlockSize};
     cuuint32_t box[3] = {64, 64, 1};
@@ -247,6 +281,7 @@ mla_status_t launch_attention(const void* q_nope, const void* q_pe, const void* 
     cuuint64_t strides[3] = {(cuuint64_t)mla::kDQK * 2, 128, (cuuint64_t)mla::kDQK * 2 * mla::kBlockSize};
     cuuint32_t box[4] = {64, 64, 2, 1};
     if (!encode(&tm_kv2, kv_cache, 4, dims, strides, box)) return MLA_ERR_INVALID_ARG;
+    }
   }
   {
     cuuint64_t dims[2] = {(cuuint64_t)mla::kDLatent, (cuuint64_t)rows};
@@ -277,7 +312,8 @@ mla_status_t launch_attention(const void* q_nope, const void* q_pe, const void* 
     if (!encode(&tm_part, part_o, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
       return MLA_ERR_INVALID_ARG;
   }
-  if (mla::launch_decode(tm_kv, tm_kv2, tm_qn, tm_qp, tm_out, tm_part, block_table, max_blocks, cache_seqlens,
+  if (mla::launch_decode(fp8, tm_kv, tm_kv2, fp8 ? &tm_kpe : nullptr, fp8 ? &tm_scl : nullptr, tm_qn, tm_qp,
+                         tm_out, tm_part, block_table, max_blocks, cache_seqlens,
                          q_lens, static_cast<const int32_t*>(metadata), num_blocks, B, s_q, H, softmax_scale,
                          causal != 0,
                          out, lse, part_o, part_lse, status, 2 * g.P * g.T, g_wait_timeout_ns.load(), g_inject_stall.load(), s) != cudaSuccess)
@@ -299,8 +335,8 @@ mla_status_t mla_decode_attention(const void* q_nope, const void* q_pe, const vo
                                       B, s_q, H, softmax_scale, metadata, metadata_bytes, workspace,
                                       workspace_bytes, out, lse, status, &g);
   if (st != MLA_OK) return st;
-  return launch_attention(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, nullptr, B,
-                          s_q, H, softmax_scale, causal, metadata, workspace, out, lse, status, g,
+  return launch_attention(false, q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens,
+                          nullptr, B, s_q, H, softmax_scale, causal, metadata, workspace, out, lse, status, g,
                           static_cast<cudaStream_t>(stream));
 }
 
@@ -344,11 +380,16 @@ mla_status_t mla_decode(const void* q_nope, const void* q_pe, const void* kv_cac
                            lse, status, stream);
 }
 
-mla_status_t mla_decode_ragged(const void* q_nope, const void* q_pe, const void* kv_cache, int64_t num_blocks,
-                               const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
-                               const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
-                               const void* metadata, size_t metadata_bytes, void* workspace,
-                               size_t workspace_bytes, void* out, float* lse, int32_t* status, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Validation, attention and combine launches shared by the bf16 and FP8 entry points.
+mla_status_t decode_any(bool fp8, const void* q_nope, const void* q_pe, const void* kv_cache, int64_t num_blocks,
+                        const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                        const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
+                        const void* metadata, size_t metadata_bytes, void* workspace, size_t workspace_bytes,
+                        void* out, float* lse, int32_t* status, void* stream) {
   if (q_lens && (reinterpret_cast<uintptr_t>(q_lens) & 3u)) return MLA_ERR_INVALID_ARG;
   DecodeGeom g;
   mla_status_t st = check_decode_args(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens,
@@ -356,8 +397,8 @@ mla_status_t mla_decode_ragged(const void* q_nope, const void* q_pe, const void*
                                       workspace_bytes, out, lse, status, &g);
   if (st != MLA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_attention(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, q_lens, B, s_q,
-                        H, softmax_scale, causal, metadata, workspace, out, lse, status, g, s);
+  st = launch_attention(fp8, q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, q_lens, B,
+                        s_q, H, softmax_scale, causal, metadata, workspace, out, lse, status, g, s);
   if (st != MLA_OK) return st;
   const float* part_o = static_cast<const float*>(workspace);
   const float* part_lse = part_o + g.slots * g.M * mla::kDLatent;
@@ -365,6 +406,47 @@ mla_status_t mla_decode_ragged(const void* q_nope, const void* q_pe, const void*
                           g.P, part_o, part_lse, out, lse, s) != cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status_t mla_decode_ragged(const void* q_nope, const void* q_pe, const void* kv_cache, int64_t num_blocks,
+                               const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                               const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
+                               const void* metadata, size_t metadata_bytes, void* workspace,
+                               size_t workspace_bytes, void* out, float* lse, int32_t* status, void* stream) {
+  return decode_any(false, q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, q_lens, B,
+                    s_q, H, softmax_scale, causal, metadata, metadata_bytes, workspace, workspace_bytes, out, lse,
+                    status, stream);
+}
+
+mla_status_t mla_decode_fp8(const void* q_nope, const void* q_pe, const void* kv_fp8, int64_t num_blocks,
+                            const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                            const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
+                            const void* metadata, size_t metadata_bytes, void* workspace, size_t workspace_bytes,
+                            void* out, float* lse, int32_t* status, void* stream) {
+  return decode_any(true, q_nope, q_pe, kv_fp8, num_blocks, block_table, max_blocks, cache_seqlens, q_lens, B,
+                    s_q, H, softmax_scale, causal, metadata, metadata_bytes, workspace, workspace_bytes, out, lse,
+                    status, stream);
+}
+
+mla_status_t mla_decode_fp8_attention(const void* q_nope, const void* q_pe, const void* kv_fp8, int64_t num_blocks,
+                                      const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                                      const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
+                                      const void* metadata, size_t metadata_bytes, void* workspace,
+                                      size_t workspace_bytes, void* out, float* lse, int32_t* status,
+                                      void* stream) {
+  if (q_lens && (reinterpret_cast<uintptr_t>(q_lens) & 3u)) return MLA_ERR_INVALID_ARG;
+  DecodeGeom g;
+  mla_status_t st = check_decode_args(q_nope, q_pe, kv_fp8, num_blocks, block_table, max_blocks, cache_seqlens,
+                                      B, s_q, H, softmax_scale, metadata, metadata_bytes, workspace,
+                                      workspace_bytes, out, lse, status, &g);
+  if (st != MLA_OK) return st;
+  return launch_attention(true, q_nope, q_pe, kv_fp8, num_blocks, block_table, max_blocks, cache_seqlens, q_lens,
+                          B, s_q, H, softmax_scale, causal, metadata, workspace, out, lse, status, g,
+                          static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

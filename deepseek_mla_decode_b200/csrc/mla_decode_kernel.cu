@@ -19,18 +19,26 @@
 //       all 256 dims of that half.
 // O uses TMEM columns [0, 256), the two S buffers [256, 384) and [384, 512).
 //
-// Warp roles (448 threads): warps 0, 2, 3, 13 = TMA producers (stage k is issued by
-// producer k % 4), warp 1 = MMA issuer (leader CTA only) and TMEM owner, warps 4..11 =
-// softmax / correction / epilogue (thread = one row x 64 keys of S, one row x 128 dims
-// of O), warp 12 = Q loader.
-// Every mbarrier wait is bounded; a timeout sets MLA_DEVICE_ERR_TIMEOUT and raises a
-// CTA-wide abort flag; every role then stops issuing at its next wait (decisions that
-// several warps share go through one barrier, so they leave together), the pair drains
-// its asynchronous work and the kernel returns.
+// Cache formats: the bf16 cache ([block][64][576] bf16) is staged by TMA straight into
+// the ring the MMAs read.  The FP8 cache (656-byte rows: e4m3 codes of c_kv / scale,
+// bf16 k_pe / scale, fp32 scale; the row format of mla_fp8.cu) is staged by TMA into a
+// separate ring of raw bytes, and converter warps turn each stage into the same bf16
+// ring slot the bf16 path would have loaded.  The codes convert to bf16 exactly (their
+// values are the e4m3 values); the per-key scale multiplies the scores (S = scale * S')
+// and the weights that enter PV (P' = bf16(e * scale)), and the row sums stay in the
+// unscaled weights e.
+//
+// Warp roles, bf16 cache (384 threads): warps 0, 2, 3 = TMA producers (ring stage k is
+// issued by producer k % 3; warp 0 also loads Q), warp 1 = MMA issuer (leader CTA only)
+// and TMEM owner, warps 4..11 = softmax / correction / epilogue (thread = one row x 64
+// keys of S, one row x 128 dims of O).  FP8 cache (512 threads): the same, plus warps
+// 12..15 = converters; setmaxnreg moves registers from the producer/MMA and converter
+// warpgroups to the softmax warpgroups.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <cstring>
 #include "mla_internal.h"
 #include "ptx_sm100.cuh"
 
@@ -40,13 +48,14 @@ using namespace ptx;
 
 namespace {
 
-constexpr int kNumThreads = 384;  // 12 warps: 3 per SM sub-partition, 168 registers per thread
 constexpr int kNumProducers = 3;  // warps 0, 2, 3 (warp 0 also loads Q)
 constexpr int kMmaWarp = 1;
 constexpr int kSoftmaxWarp0 = 4;   // warps 4..11
 constexpr int kNumSoftmaxThreads = 256;
-constexpr int kStages = 7;
-constexpr int kStageBytes = 16384;
+constexpr int kConvWarp0 = 12;     // FP8 cache: warps 12..15
+constexpr int kNumConvThreads = 128;
+constexpr int kMaxStages = 7;
+constexpr int kStageBytes = 16384;  // one bf16 ring slot
 constexpr int kChunkBytes = 8192;  // one 64-row x 64-column bf16 SW128 box
 constexpr int kQChunks = 9;        // 576 / 64
 constexpr int kQBytes = kQChunks * kChunkBytes;
@@ -54,18 +63,49 @@ constexpr int kPBytes = 4 * kChunkBytes;  // 64 rows x 256 keys bf16
 constexpr int kSmemQ = 0;
 constexpr int kSmemP = kSmemQ + kQBytes;
 constexpr int kSmemRing = kSmemP + kPBytes;
-constexpr int kSmemDyn = kSmemRing + kStages * kStageBytes;
+// FP8 cache: raw stages of 8 KB (an e4m3 slab or one block of scaled k_pe) and two
+// buffers of per-key scales (4 blocks x 64 rows x 16 bytes, the scale in the first 4)
+constexpr int kStgBytes = 8192;
+constexpr int kMaxStg = 8;
+constexpr int kScaleBufBytes = 4096;
+constexpr int kSlabBlockBytes = 64 * 64;           // one block's 64-column slab of codes
+constexpr int kScaleBlockBytes = 64 * 16;          // one block's scales (16 bytes per row)
+constexpr int kStgPerQk = 8 + 2;                   // raw stages per tile for QK
+// FP8 kernel register split (setmaxnreg, per warpgroup): warps 0-3 (producers, MMA),
+// 4-11 (softmax), 12-15 (converters); 128 x (issue + conv) + 256 x softmax must equal
+// the 512 x 128 registers the block is launched with.
+constexpr int kRegsIssue = 88, kRegsConv = 72, kRegsSoftmax = 176;
+static_assert(128 * (kRegsIssue + kRegsConv) + 256 * kRegsSoftmax == 512 * 128, "register split");
+
+template <bool kFp8>
+struct Cfg {
+  static constexpr int kThreads = kFp8 ? 512 : 384;
+  static constexpr int kStages = kFp8 ? 3 : 7;  // bf16 ring slots
+  static constexpr int kStg = kFp8 ? 7 : 0;     // raw FP8 stages
+  static constexpr int kSmemStg = kSmemRing + kStages * kStageBytes;
+  static constexpr int kSmemScale = kSmemStg + kStg * kStgBytes;
+  static constexpr int kSmemDyn = kSmemScale + (kFp8 ? 2 * kScaleBufBytes : 0);
+  static_assert(kStages <= kMaxStages && kStg <= kMaxStg, "ring sizes");
+};
 constexpr uint32_t kTmemO = 0, kTmemS0 = 256, kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only when the max grows by > 2^8
 constexpr uint32_t kIdescQK = make_idesc_bf16(128, 256, false, false);
 constexpr uint32_t kIdescPV = make_idesc_bf16(128, 256, false, true);
 constexpr int kBarSoftmax = 1;  // named barrier id for the 256 softmax threads
+constexpr int kBarConv = 2;     // named barrier id for the 128 converter threads
 constexpr uint64_t kDrainWaitNs = 100000000ull;  // bound on the post-abort wait for tensor-core work
 constexpr uint64_t kQuiesceNs = 500000ull;       // post-abort wait for TMA loads in flight
 
 struct Params {
-  CUtensorMap tm_kv;   // [num_blocks][64][576] bf16, box {64, 64, 1}, SW128
-  CUtensorMap tm_kv2;  // same memory as [num_blocks][9][64][64], box {64, 64, 2, 1}, SW128
+  // bf16 cache: tm_kv = [num_blocks][64][576] bf16, box {64, 64, 1}, SW128; tm_kv2 = the
+  // same memory as [num_blocks][9][64][64], box {64, 64, 2, 1}, SW128.
+  // FP8 cache: tm_kv = the packed rows as bytes [num_blocks][64][656], box {64, 64, 1}
+  // (one 64-column slab of codes, no swizzle); tm_kv2 = the same bytes, box {128, 64, 1},
+  // SW128 (a 128-column slab for PV).
+  CUtensorMap tm_kv;
+  CUtensorMap tm_kv2;
+  CUtensorMap tm_kpe;   // FP8 cache: rows as [num_blocks][64][328] bf16, box {64, 64, 1} at column 256, SW128
+  CUtensorMap tm_scl;   // FP8 cache: rows as [num_blocks][64][164] fp32, box {4, 64, 1} at column 160
   CUtensorMap tm_qn;  // [B*M][512] bf16, box {64, 64}, SW128
   CUtensorMap tm_qp;  // [B*M][64] bf16, box {64, 64}, SW128
   CUtensorMap tm_out;   // out as [B][M][512] bf16, box {64, 64, 1}, SW128 (TMA store)
@@ -89,8 +129,13 @@ struct Params {
 };
 
 struct __align__(8) Ctrl {
-  uint64_t full[kStages];   // leader: stage landed in both CTAs (count 1 + tx of both CTAs)
-  uint64_t empty[kStages];  // both: stage consumed by the MMAs (commit)
+  uint64_t full[kMaxStages];   // leader: stage landed in both CTAs (bf16: count 1 + tx of both
+                               // CTAs; FP8: count 2, one converter arrival per CTA)
+  uint64_t empty[kMaxStages];  // both: stage consumed by the MMAs (commit)
+  uint64_t stg_full[kMaxStg];  // FP8, both: raw stage landed (count 1 + tx)
+  uint64_t stg_empty[kMaxStg]; // FP8, both: raw stage read by the converters (count 1)
+  uint64_t sc_full[2];         // FP8, both: scales of a tile landed (count 1 + tx)
+  uint64_t sc_empty[2];        // FP8, both: scales of a tile used by the softmax (count 1)
   uint64_t q_full;          // leader: Q of both CTAs landed (count 1 + tx)
   uint64_t q_empty;         // both: last QK of the piece done (commit)
   uint64_t s_full[2];       // both: S buffer written (commit)
@@ -194,20 +239,13 @@ __device__ __forceinline__ void set_status(const Params& p, int bits) {
 }
 
 // Bounded wait that also gives up when another role of this CTA aborted.
-// cluster_scope selects acquire.cluster, needed only where the peer CTA's generic
-// shared-memory writes (P) or TMEM reads are published by a
-// release.cluster arrive; data landed by TMA is ordered by its transaction bytes and
-// a CTA-scope wait suffices (the cluster-scope acquire costs ~0.4 us per wait).
-__device__ __forceinline__ bool wait_bar(Ctrl* c, const Params& p, uint32_t bar, uint32_t parity,
-                                         bool cluster_scope) {
-  const bool ok0 = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
-  if (ok0) return true;
+__device__ __forceinline__ bool wait_bar(Ctrl* c, const Params& p, uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
   for (;;) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i) {
-      const bool ok = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
-      if (ok) return true;
+      if (mbar_try_wait(bar, parity)) return true;
     }
     if (c->abort) return false;
     if (globaltimer_ns() > deadline) {
@@ -321,6 +359,42 @@ __device__ __forceinline__ float add_bf16x2_to(float acc, uint32_t v) {
   return r;
 }
 
+// ---- FP8 cache helpers --------------------------------------------------------
+// TMA load into this CTA's own shared memory, completing on its own barrier.
+__device__ __forceinline__ void tma_load_3d_if(bool on, uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1,
+                                               int c2) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %6, 0;\n\t"
+      "@q cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];\n\t}" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"((uint32_t)on)
+      : "memory");
+}
+template <int kRegs>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <int kRegs>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+// Two e4m3 codes (bytes b0, b1 of w, or b2, b3 with kHigh) -> two bf16 of the same
+// values, exactly.  Per 16-bit lane a byte permute builds [sign of the code replicated |
+// code]; shifting left by 4 and masking leaves sign at bit 15, the code's 4 exponent
+// bits at 10..7 and its 3 mantissa bits at 6..4: a bf16 pattern whose exponent field is
+// the e4m3 exponent field, i.e. the code's value times 2^(7 - 127) for normal codes and,
+// through the bf16 subnormal range, for subnormal codes and zero too.  One bf16 multiply
+// by 2^120 (exact: every result is a normal bf16) restores the value.
+template <bool kHigh>
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t w) {
+  uint32_t a;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(a) : "r"(w), "n"(kHigh ? 0xB3A2 : 0x9180));
+  const uint32_t t = (a << 4) & 0x87F087F0u;
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(t), "r"(0x7B807B80u));  // 2^120 in both lanes
+  return r;
+}
+
 __device__ __forceinline__ int clamp_block_id(const Params& p, int32_t id) {
   if (id < 0 || (int64_t)id >= p.num_blocks) {
     set_status(p, kErrBlockId);
@@ -362,13 +436,17 @@ __device__ __forceinline__ void write_orphan_rows(const Params& p, int part, int
 // ===========================================================================
 // the kernel
 // ===========================================================================
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
+template <bool kFp8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     mla_decode_kernel(const __grid_constant__ Params p) {
+  using C = Cfg<kFp8>;
+  constexpr int kStages = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ Ctrl ctrl;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + kSmemQ, sP = sbase + kSmemP, sRing = sbase + kSmemRing;
+  const uint32_t sStg = sbase + C::kSmemStg, sScale = sbase + C::kSmemScale;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
@@ -379,8 +457,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
   // is launched as a programmatic dependent) -----------------------------------
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&ctrl.full[s]), 1);
+      mbar_init(smem_u32(&ctrl.full[s]), kFp8 ? 2 : 1);
       mbar_init(smem_u32(&ctrl.empty[s]), 1);
+    }
+    if constexpr (kFp8) {
+      for (int s = 0; s < C::kStg; ++s) {
+        mbar_init(smem_u32(&ctrl.stg_full[s]), 1);
+        mbar_init(smem_u32(&ctrl.stg_empty[s]), 1);
+      }
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(smem_u32(&ctrl.sc_full[s]), 1);
+        mbar_init(smem_u32(&ctrl.sc_empty[s]), 1);
+      }
     }
     mbar_init(smem_u32(&ctrl.q_full), 1);
     mbar_init(smem_u32(&ctrl.q_empty), 1);
@@ -409,6 +497,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     prefetch_tmap(&p.tm_qp);
     prefetch_tmap(&p.tm_out);
     prefetch_tmap(&p.tm_part);
+    if constexpr (kFp8) {
+      prefetch_tmap(&p.tm_kpe);
+      prefetch_tmap(&p.tm_scl);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -438,19 +530,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     // each piece's Q.
     // =======================================================================
     if (warp == 0 || warp == 2 || warp == 3) {
+      if constexpr (kFp8) regs_dec<kRegsIssue>();
       const int pi = (warp == 0) ? 0 : warp - 1;
       int32_t* idwin = ctrl.block_ids[pi];
       PieceWalker walk(p, part, tile_row0);
       uint32_t it = 0;
       bool ok = true;
       auto mine = [&]() { return (int)(it % kNumProducers) == pi; };
-      // acquire the ring slot of stage `it` (every lane waits, the warp stays converged)
+      // acquire the slot of stage `it` (every lane waits, the warp stays converged): a
+      // bf16 ring slot freed by the MMAs, or (FP8 cache) a raw stage freed by the
+      // converters
       auto acquire = [&](uint32_t& slot) -> bool {
-        slot = it % kStages;
-        const uint32_t use = it / kStages;
-        if (use > 0 && !wait_bar(&ctrl, p, smem_u32(&ctrl.empty[slot]), (use - 1) & 1, false)) return false;
+        constexpr int kSlots = kFp8 ? C::kStg : kStages;
+        slot = it % kSlots;
+        const uint32_t use = it / kSlots;
+        const uint32_t eb = kFp8 ? smem_u32(&ctrl.stg_empty[slot]) : smem_u32(&ctrl.empty[slot]);
+        if (use > 0 && !wait_bar(&ctrl, p, eb, (use - 1) & 1)) return false;
         return true;
       };
+      uint32_t ntile = 0;  // tiles issued so far (FP8: selects the scale buffer)
       // Physical block ids of the current piece, fetched 32 at a time (one coalesced
       // load per lane) one chunk ahead of use into this warp's 128-entry window, from
       // window offset `cur_base` on; invalid ids are clamped to block 0 here (the
@@ -469,6 +567,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           id_pending = fetch_id(32 * id_chunks + lane);
           __syncwarp();
         }
+      };
+      // FP8 cache, QK of tile t: this CTA's (up to) two blocks as 8 slabs of 64 code
+      // columns (4 KB per block), then its blocks' scaled k_pe (8 KB each, one raw stage
+      // per block, present or not); with the first slab, the scales of all the tile's
+      // blocks for the softmax.
+      auto issue_qk_fp8 = [&](int t) {
+        const int nb = blocks_in_tile(cur, t);
+        const int own0 = 2 * (int)rank;
+        ensure_ids(t * kBlocksPerTile + nb - 1);
+        const int own = min(max(nb - own0, 0), 2);
+        const int my_id = idwin[(cur_base + t * kBlocksPerTile + own0 + (lane & 1)) % kIdRing];
+        for (int st = 0; st < kStgPerQk && ok; ++st) {  // 8 code slabs, then 2 k_pe blocks
+          if (!mine()) {
+            ++it;
+            continue;
+          }
+          if (st == 0) {  // the tile's scales, into buffer ntile & 1
+            const uint32_t sb = ntile & 1, use = ntile >> 1;
+            if (use > 0)
+              ok = __shfl_sync(0xffffffffu, wait_bar(&ctrl, p, smem_u32(&ctrl.sc_empty[sb]), (use - 1) & 1), 0);
+            if (!ok) break;
+            const uint32_t fb = smem_u32(&ctrl.sc_full[sb]);
+            expect_tx_if(lane == 0, fb, nb * kScaleBlockBytes);
+            const int id = idwin[(cur_base + t * kBlocksPerTile + (lane & 3)) % kIdRing];
+            tma_load_3d_if(lane < nb, sScale + sb * kScaleBufBytes + lane * kScaleBlockBytes, &p.tm_scl, fb,
+                           kOffScale8 / 4, 0, id);
+          }
+          uint32_t slot;
+          ok = __shfl_sync(0xffffffffu, acquire(slot), 0);
+          if (!ok) break;
+          const uint32_t fb = smem_u32(&ctrl.stg_full[slot]);
+          if (st < 8) {
+            expect_tx_if(lane == 0, fb, own * kSlabBlockBytes);
+            tma_load_3d_if(lane < own, sStg + slot * kStgBytes + lane * kSlabBlockBytes, &p.tm_kv, fb, 64 * st, 0,
+                           my_id);
+          } else {
+            const int kp = st - 8;
+            const int id = idwin[(cur_base + t * kBlocksPerTile + own0 + kp) % kIdRing];
+            expect_tx_if(lane == 0, fb, kp < own ? kStgBytes : 0);
+            tma_load_3d_if(lane == 0 && kp < own, sStg + slot * kStgBytes, &p.tm_kpe, fb, kDLatent / 2, 0, id);
+          }
+          ++it;
+        }
+        ++ntile;
       };
       auto issue_qk = [&](int t) {
         const int nb = blocks_in_tile(cur, t);
@@ -522,10 +664,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
             ok = __shfl_sync(0xffffffffu, acquire(slot), 0);
             if (!ok) break;
             const int d0 = 256 * h + 128 * (int)rank;
-            const uint32_t fb = smem_u32(&ctrl.full[slot]);
-            expect_tx_if(lane == 0 && leader, fb, 2 * kStageBytes);
-            tma_load_4d_cg2_if(lane == 0, sRing + slot * kStageBytes, &p.tm_kv2, mapa_shared(fb, 0), 0,
-                               rv - kBlockSize, d0 / 64, id);
+            if constexpr (kFp8) {  // one block's 128-column slab of codes (8 KB)
+              const uint32_t fb = smem_u32(&ctrl.stg_full[slot]);
+              expect_tx_if(lane == 0, fb, kStgBytes);
+              tma_load_3d_if(lane == 0, sStg + slot * kStgBytes, &p.tm_kv2, fb, d0, rv - kBlockSize, id);
+            } else {
+              const uint32_t fb = smem_u32(&ctrl.full[slot]);
+              expect_tx_if(lane == 0 && leader, fb, 2 * kStageBytes);
+              tma_load_4d_cg2_if(lane == 0, sRing + slot * kStageBytes, &p.tm_kv2, mapa_shared(fb, 0), 0,
+                                 rv - kBlockSize, d0 / 64, id);
+            }
             ++it;
           }
         }
@@ -535,7 +683,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
       const uint32_t q_full_l = mapa_shared(smem_u32(&ctrl.q_full), 0);
       auto load_q = [&](const Piece& pc, int piece_idx) {
         if (piece_idx > 0)
-          ok = __shfl_sync(0xffffffffu, wait_bar(&ctrl, p, smem_u32(&ctrl.q_empty), (piece_idx - 1) & 1, false), 0);
+          ok = __shfl_sync(0xffffffffu, wait_bar(&ctrl, p, smem_u32(&ctrl.q_empty), (piece_idx - 1) & 1), 0);
         if (!ok) return;
         const int row_base = pc.b * p.M + tile_row0 + kRowsPerCta * (int)rank;
         expect_tx_if(lane == 0 && leader, smem_u32(&ctrl.q_full), 2 * kQBytes);
@@ -567,7 +715,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
             id_next = (lane < nxt.k_hi - nxt.k_lo) ? clamp_block_id(p, btn[nxt.k_lo + lane]) : 0;
           }
           if (t == 0 && pi == 0) load_q(cur, npieces);
-          if (ok) issue_qk(t);
+          if (ok) {
+            if constexpr (kFp8)
+              issue_qk_fp8(t);
+            else
+              issue_qk(t);
+          }
           if (ok && prv_t >= 0) issue_pv(prv, prv_base, prv_t);
           prv = cur;
           prv_base = cur_base;
@@ -592,6 +745,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     // MMA issuer (leader CTA only)
     // =======================================================================
     else if (warp == kMmaWarp && leader) {
+      if constexpr (kFp8) regs_dec<kRegsIssue>();
       // Every lane waits and the elected lane's predicate issues.  No full-warp
       // collective sits inside the loop, so lanes that leave it at different points
       // after a wait ran out cannot deadlock the warp; they meet again at teardown.
@@ -619,7 +773,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
         const uint32_t buf = qk_count & 1;
         const uint32_t d = tmem + kTmemS0 + 128 * buf;
         for (int c = 0; c < kQChunks && ok; ++c) {
-          ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), phase, false);
+          ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), phase);
           if (!ok) break;
           const uint64_t a0 = dq0 + c * kChunkD, b0 = dk0 + slot * kStageD;
 #pragma unroll
@@ -636,14 +790,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
       // PV of tile t of piece pc, the piece_idx-th piece of this partition
       auto mma_pv = [&](const Piece& pc, int piece_idx, int t) {
         if (!ok) return;
-        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_full), pv_count & 1, true);
-        if (ok && t == 0 && piece_idx > 0) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.o_free), (piece_idx - 1) & 1, true);
+        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_full), pv_count & 1);
+        if (ok && t == 0 && piece_idx > 0) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.o_free), (piece_idx - 1) & 1);
         if (!ok) return;
         tc_fence_after();
         const int nb = blocks_in_tile(pc, t);
         for (int h = 0; h < 2 && ok; ++h) {
           for (int kb = 0; kb < nb && ok; ++kb) {
-            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), phase, false);
+            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[slot]), phase);
             if (!ok) break;
             // the sequence's last block sits in rows [64 - rv, 64): skip whole zero steps
             const int rv = rows_in_block(pc, t, kb);
@@ -664,9 +818,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
       // same ring order as the producers: QK of each tile, then PV of the tile before
       Piece cur, prv{};
       int prv_t = -1, prv_idx = 0;
-      if (p.inject_stall) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.never), 0, false);
+      if (p.inject_stall) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.never), 0);
       while (ok && walk.next(cur)) {
-        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.q_full), npieces & 1, false);
+        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.q_full), npieces & 1);
         const int nt = num_tiles(cur);
         for (int t = 0; t < nt && ok; ++t) {
           mma_qk(nt, t);
@@ -683,6 +837,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
     // softmax / correction / epilogue
     // =======================================================================
     else if (warp >= kSoftmaxWarp0 && warp < kSoftmaxWarp0 + 8) {
+      if constexpr (kFp8) regs_inc<kRegsSoftmax>();
       const int st = tid - kSoftmaxWarp0 * 32;  // 0..255
       const int g = st >> 7;                   // column group: keys 64g.. of each half; O half g
       const int L = st & 127;                  // TMEM lane
@@ -807,7 +962,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           const uint32_t buf = qk_count & 1;
           // A wait that runs out does not leave the loop here: the thread carries on to
           // the next AND barrier, which makes all 256 threads leave together.
-          ok = wait_bar(&ctrl, p, smem_u32(&ctrl.s_full[buf]), (qk_count >> 1) & 1, false) && ok;
+          ok = wait_bar(&ctrl, p, smem_u32(&ctrl.s_full[buf]), (qk_count >> 1) & 1) && ok;
+          // FP8 cache: the tile's per-key scales (key 64 j + c of the tile at float
+          // 256 j + 4 c of its buffer); this thread's 64 keys are block 2 hk + g
+          const float* scb = reinterpret_cast<const float*>(smem + C::kSmemScale + (qk_count & 1) * kScaleBufBytes +
+                                                            (2 * hk + g) * kScaleBlockBytes);
+          if constexpr (kFp8)
+            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.sc_full[qk_count & 1]), (qk_count >> 1) & 1) && ok;
           tc_fence_after();
           uint32_t sr[64];
           {
@@ -827,6 +988,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           // Row maximum of the raw scores (the scale is positive, so it keeps their
           // order), over four independent chains.
           float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+          const float sl2 = p.scale_log2;
+          if constexpr (kFp8) {
+            // scores in log2 units, x = S' * scale_key * scale_log2, kept in sr
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+              const float x = __uint_as_float(sr[c]) * (scb[4 * c] * sl2);
+              sr[c] = __float_as_uint(x);
+            }
+          }
           if (full) {
 #pragma unroll
             for (int c = 0; c < 64; c += 4) {
@@ -844,7 +1014,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
               if (c + 3 < cnt) mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
             }
           }
-          const float lmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+          const float lmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * (kFp8 ? 1.0f : sl2);
           ctrl.red_max[qk_count & 1][2 * hk + g][m] = lmax;
           go = named_bar_and(kBarSoftmax, kNumSoftmaxThreads, ok);
           if (!go) break;
@@ -862,40 +1032,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
             l32_part *= alpha;
           }
           const float nref = (m_used == -INFINITY) ? 0.f : -m_used;
-          const float sl2 = p.scale_log2;
           uint32_t pk[32];
-          // weights 2^(s * scale_log2 - m); sums of the bf16-rounded weights (output
-          // normaliser) and of the fp32 weights (lse), two chains each
+          // bf16 cache: weights 2^(s * scale_log2 - m); sums of the bf16-rounded weights
+          // (output normaliser) and of the fp32 weights (lse), two chains each
           float ls0 = 0.f, ls1 = 0.f, lf0 = 0.f, lf1 = 0.f;
-          if (full) {
+          if constexpr (kFp8) {
+            // weights e = 2^(x - m) (their fp32 sums normalise the output and give the
+            // lse); the PV operand is P' = bf16(e * scale_key), since V = scale_key * codes
 #pragma unroll
-            for (int c = 0; c < 64; c += 4) {
-              const float e0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, nref));
-              const float e1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, nref));
-              const float e2 = fast_exp2(fmaf(__uint_as_float(sr[c + 2]), sl2, nref));
-              const float e3 = fast_exp2(fmaf(__uint_as_float(sr[c + 3]), sl2, nref));
-              const uint32_t v0 = pack_bf16x2(e0, e1), v1 = pack_bf16x2(e2, e3);
-              pk[c >> 1] = v0;
-              pk[(c >> 1) + 1] = v1;
-              ls0 = add_bf16x2_to(ls0, v0);
-              ls1 = add_bf16x2_to(ls1, v1);
-              lf0 += e0 + e1;
-              lf1 += e2 + e3;
+            for (int c = 0; c < 64; c += 2) {
+              const bool v0 = full || c < cnt, v1 = full || c + 1 < cnt;
+              const float e0 = v0 ? fast_exp2(__uint_as_float(sr[c]) + nref) : 0.f;
+              const float e1 = v1 ? fast_exp2(__uint_as_float(sr[c + 1]) + nref) : 0.f;
+              const float p0 = v0 ? e0 * scb[4 * c] : 0.f;
+              const float p1 = v1 ? e1 * scb[4 * c + 4] : 0.f;
+              pk[c >> 1] = pack_bf16x2(p0, p1);
+              if (c & 2)
+                lf1 += e0 + e1;
+              else
+                lf0 += e0 + e1;
             }
+            ls0 = lf0;
+            ls1 = lf1;
           } else {
+            if (full) {
 #pragma unroll
-            for (int c = 0; c < 64; c += 4) {
-              const float e0 = (c < cnt) ? fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, nref)) : 0.f;
-              const float e1 = (c + 1 < cnt) ? fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, nref)) : 0.f;
-              const float e2 = (c + 2 < cnt) ? fast_exp2(fmaf(__uint_as_float(sr[c + 2]), sl2, nref)) : 0.f;
-              const float e3 = (c + 3 < cnt) ? fast_exp2(fmaf(__uint_as_float(sr[c + 3]), sl2, nref)) : 0.f;
-              const uint32_t v0 = pack_bf16x2(e0, e1), v1 = pack_bf16x2(e2, e3);
-              pk[c >> 1] = v0;
-              pk[(c >> 1) + 1] = v1;
-              ls0 = add_bf16x2_to(ls0, v0);
-              ls1 = add_bf16x2_to(ls1, v1);
-              lf0 += e0 + e1;
-              lf1 += e2 + e3;
+              for (int c = 0; c < 64; c += 4) {
+                const float e0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, nref));
+                const float e1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, nref));
+                const float e2 = fast_exp2(fmaf(__uint_as_float(sr[c + 2]), sl2, nref));
+                const float e3 = fast_exp2(fmaf(__uint_as_float(sr[c + 3]), sl2, nref));
+                const uint32_t v0 = pack_bf16x2(e0, e1), v1 = pack_bf16x2(e2, e3);
+                pk[c >> 1] = v0;
+                pk[(c >> 1) + 1] = v1;
+                ls0 = add_bf16x2_to(ls0, v0);
+                ls1 = add_bf16x2_to(ls1, v1);
+                lf0 += e0 + e1;
+                lf1 += e2 + e3;
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 64; c += 4) {
+                const float e0 = (c < cnt) ? fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, nref)) : 0.f;
+                const float e1 = (c + 1 < cnt) ? fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, nref)) : 0.f;
+                const float e2 = (c + 2 < cnt) ? fast_exp2(fmaf(__uint_as_float(sr[c + 2]), sl2, nref)) : 0.f;
+                const float e3 = (c + 3 < cnt) ? fast_exp2(fmaf(__uint_as_float(sr[c + 3]), sl2, nref)) : 0.f;
+                const uint32_t v0 = pack_bf16x2(e0, e1), v1 = pack_bf16x2(e2, e3);
+                pk[c >> 1] = v0;
+                pk[(c >> 1) + 1] = v1;
+                ls0 = add_bf16x2_to(ls0, v0);
+                ls1 = add_bf16x2_to(ls1, v1);
+                lf0 += e0 + e1;
+                lf1 += e2 + e3;
+              }
             }
           }
           l_part += ls0 + ls1;
@@ -903,7 +1092,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
           // PV of the previous tile (possibly the previous piece's last) must be done
           // before P is overwritten, O is rescaled or the previous piece's O is read.
           if (qk_count >= 1) {
-            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1, false) && ok;
+            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1) && ok;
             ++pv_count;
             tc_fence_after();
             if (t == 0) {
@@ -976,6 +1165,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
               mbar_arrive(smem_u32(&ctrl.p_full));
             else
               mbar_arrive_remote(p_full_l);
+            if constexpr (kFp8) mbar_arrive(smem_u32(&ctrl.sc_empty[qk_count & 1]));  // scales read
           }
           ++qk_count;
         }
@@ -1004,11 +1194,149 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
       // the last piece's epilogue, after its last PV (the AND makes the decision uniform)
       go = named_bar_and(kBarSoftmax, kNumSoftmaxThreads, ok && go);
       if (go && pend) {
-        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1, false) && ok;
+        ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1) && ok;
         ++pv_count;
         tc_fence_after();
         epilogue();
       }
+    }
+    // =======================================================================
+    // FP8 cache: converters (warps 12..15).  In ring order, each raw stage becomes a
+    // bf16 ring slot in exactly the layout the bf16 path's TMA would have produced
+    // (64-column K-major boxes for QK, 2 x 64-column boxes for PV, 128-byte swizzle),
+    // then both CTAs' converters arrive on the leader's full barrier of that slot.
+    // =======================================================================
+    else if (warp >= kConvWarp0) {
+      if constexpr (kFp8) {
+        regs_dec<kRegsConv>();
+        constexpr int kStg = C::kStg;
+        const int ct = tid - kConvWarp0 * 32;  // 0..127
+        PieceWalker walk(p, part, tile_row0);
+        uint32_t js = 0, ir = 0;  // raw stages and ring slots consumed so far
+        bool ok = true, go = true;
+        auto wait_raw = [&](uint32_t j) {
+          ok = wait_bar(&ctrl, p, smem_u32(&ctrl.stg_full[j % kStg]), (j / kStg) & 1) && ok;
+        };
+        auto wait_slot = [&]() {
+          if (ir >= (uint32_t)kStages)
+            ok = wait_bar(&ctrl, p, smem_u32(&ctrl.empty[ir % kStages]), ((ir / kStages) - 1) & 1) && ok;
+        };
+        // Hand slot ir to the MMAs and raw stages [j0, j0 + nraw) back to the
+        // producers.  The AND barrier makes a timed-out wait leave all 128 threads
+        // together.
+        auto publish = [&](uint32_t j0, int nraw) -> bool {
+          fence_proxy_async_smem();
+          go = named_bar_and(kBarConv, kNumConvThreads, ok);
+          if (!go) return false;
+          if (ct == 0) {
+            for (int k = 0; k < nraw; ++k) mbar_arrive(smem_u32(&ctrl.stg_empty[(j0 + k) % kStg]));
+            const uint32_t fb = smem_u32(&ctrl.full[ir % kStages]);
+            if (leader)
+              mbar_arrive(fb);
+            else
+              mbar_arrive_remote(mapa_shared(fb, 0));
+          }
+          ++ir;
+          return true;
+        };
+        // QK slab: raw = box b (own block b) as [64 rows][64 codes]; slot = box b as
+        // [64 rows][128 B] swizzled.  Unit u = 16 codes: b = u >> 8, row m, granule k.
+        // Eight consecutive threads cover two rows x four granules: 128 contiguous raw
+        // bytes and eight distinct swizzled granules, so neither side has bank conflicts.
+        auto conv_slab = [&](const uint8_t* src, uint8_t* dst, int own) {
+#pragma unroll 2
+          for (int i = 0; i < 4; ++i) {
+            const int u = ct + kNumConvThreads * i, b = u >> 8;
+            if (b >= own) continue;
+            const int m = (u >> 2) & 63, k = u & 3;
+            const uint4 v = *reinterpret_cast<const uint4*>(src + b * kSlabBlockBytes + m * 64 + 16 * k);
+            uint8_t* row = dst + b * kChunkBytes + m * 128;
+            const int g0 = (2 * k) ^ (m & 7);
+            *reinterpret_cast<uint4*>(row + (g0 << 4)) =
+                make_uint4(e4m3x2_to_bf16x2<false>(v.x), e4m3x2_to_bf16x2<true>(v.x), e4m3x2_to_bf16x2<false>(v.y),
+                           e4m3x2_to_bf16x2<true>(v.y));
+            *reinterpret_cast<uint4*>(row + ((g0 ^ 1) << 4)) =
+                make_uint4(e4m3x2_to_bf16x2<false>(v.z), e4m3x2_to_bf16x2<true>(v.z), e4m3x2_to_bf16x2<false>(v.w),
+                           e4m3x2_to_bf16x2<true>(v.w));
+          }
+        };
+        // PV slab: raw = [64 rows][128 codes] swizzled; slot = two [64 rows][128 B]
+        // swizzled boxes (columns 0..63, 64..127).  Unit u: row m = u & 63, 16-column
+        // granule k = u >> 6; eight consecutive threads take eight rows of one granule.
+        auto conv_vslab = [&](const uint8_t* src, uint8_t* dst) {
+#pragma unroll 2
+          for (int i = 0; i < 4; ++i) {
+            const int u = ct + kNumConvThreads * i;
+            const int m = u & 63, k = u >> 6;
+            const uint4 v = *reinterpret_cast<const uint4*>(src + m * 128 + ((k ^ (m & 7)) << 4));
+            uint8_t* row = dst + (k >> 2) * kChunkBytes + m * 128;
+            const int g0 = (2 * (k & 3)) ^ (m & 7);
+            *reinterpret_cast<uint4*>(row + (g0 << 4)) =
+                make_uint4(e4m3x2_to_bf16x2<false>(v.x), e4m3x2_to_bf16x2<true>(v.x), e4m3x2_to_bf16x2<false>(v.y),
+                           e4m3x2_to_bf16x2<true>(v.y));
+            *reinterpret_cast<uint4*>(row + ((g0 ^ 1) << 4)) =
+                make_uint4(e4m3x2_to_bf16x2<false>(v.z), e4m3x2_to_bf16x2<true>(v.z), e4m3x2_to_bf16x2<false>(v.w),
+                           e4m3x2_to_bf16x2<true>(v.w));
+          }
+        };
+        uint8_t* const ring = smem + kSmemRing;
+        const uint8_t* const raw = smem + C::kSmemStg;
+        auto conv_qk = [&](const Piece& pc, int t) {
+          const int own = min(max(blocks_in_tile(pc, t) - 2 * (int)rank, 0), 2);
+          for (int c = 0; c < 8; ++c) {
+            wait_raw(js);
+            wait_slot();
+            if (ok) conv_slab(raw + (js % kStg) * kStgBytes, ring + (ir % kStages) * kStageBytes, own);
+            if (!publish(js, 1)) return;
+            ++js;
+          }
+          // k_pe: the two blocks' raw stages already hold the slot's boxes; copy them
+          wait_raw(js);
+          wait_raw(js + 1);
+          wait_slot();
+          if (ok) {
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+              if (b >= own) continue;
+              const uint4* src = reinterpret_cast<const uint4*>(raw + ((js + b) % kStg) * kStgBytes);
+              uint4* dst = reinterpret_cast<uint4*>(ring + (ir % kStages) * kStageBytes + b * kChunkBytes);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) dst[ct + kNumConvThreads * i] = src[ct + kNumConvThreads * i];
+            }
+          }
+          if (!publish(js, 2)) return;
+          js += 2;
+        };
+        auto conv_pv = [&](const Piece& pc, int t) {
+          const int nb = blocks_in_tile(pc, t);
+          for (int h = 0; h < 2; ++h) {
+            for (int kb = 0; kb < nb; ++kb) {
+              wait_raw(js);
+              wait_slot();
+              if (ok) conv_vslab(raw + (js % kStg) * kStgBytes, ring + (ir % kStages) * kStageBytes);
+              if (!publish(js, 1)) return;
+              ++js;
+            }
+          }
+        };
+        // the producers' and the MMAs' ring order
+        Piece cur, prv{};
+        int prv_t = -1;
+        while (go && walk.next(cur)) {
+          const int nt = num_tiles(cur);
+          for (int t = 0; t < nt && go; ++t) {
+            conv_qk(cur, t);
+            if (go && prv_t >= 0) conv_pv(prv, prv_t);
+            prv = cur;
+            prv_t = t;
+          }
+        }
+        if (go && prv_t >= 0) conv_pv(prv, prv_t);
+      }
+    }
+    // the peer CTA's MMA warp has no role; it joins its warpgroup's register release
+    else if (warp == kMmaWarp) {
+      if constexpr (kFp8) regs_dec<kRegsIssue>();
     }
   }
 
@@ -1052,16 +1380,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNumThreads, 1)
 
 }  // namespace
 
-struct DecodeLaunch {
-  CUtensorMap tm_kv, tm_qn, tm_qp;
-};
-
 cudaError_t decode_kernel_setup(int device) {
   (void)device;
-  return cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDyn + 1024);
+  cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg<false>::kSmemDyn + 1024);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(mla_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Cfg<true>::kSmemDyn + 1024);
 }
 
-cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
+// tm_kpe / tm_scl: FP8 cache only (null for the bf16 cache, which fp8 = false selects).
+cudaError_t launch_decode(bool fp8, const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
+                          const CUtensorMap* tm_kpe, const CUtensorMap* tm_scl,
                           const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
                           const CUtensorMap& tm_out, const CUtensorMap& tm_part,
                           const int32_t* block_table, int max_blocks, const int32_t* seqlens,
@@ -1069,9 +1399,15 @@ cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
                           int H, float scale, int causal, void* out, float* lse, float* part_o, float* part_lse,
                           int32_t* status, int num_ctas, uint64_t wait_timeout_ns, int inject_stall,
                           cudaStream_t stream) {
+  if (fp8 && (!tm_kpe || !tm_scl)) return cudaErrorInvalidValue;
   Params prm;
+  std::memset(&prm, 0, sizeof(prm));
   prm.tm_kv = tm_kv;
   prm.tm_kv2 = tm_kv2;
+  if (fp8) {
+    prm.tm_kpe = *tm_kpe;
+    prm.tm_scl = *tm_scl;
+  }
   prm.tm_qn = tm_qn;
   prm.tm_qp = tm_qp;
   prm.tm_out = tm_out;
@@ -1100,15 +1436,16 @@ cudaError_t launch_decode(const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
   // any input.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_ctas);
-  cfg.blockDim = dim3(kNumThreads);
-  cfg.dynamicSmemBytes = kSmemDyn + 1024;
+  cfg.blockDim = dim3(fp8 ? Cfg<true>::kThreads : Cfg<false>::kThreads);
+  cfg.dynamicSmemBytes = (fp8 ? Cfg<true>::kSmemDyn : Cfg<false>::kSmemDyn) + 1024;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mla_decode_kernel, prm);
+  return fp8 ? cudaLaunchKernelEx(&cfg, mla_decode_kernel<true>, prm)
+             : cudaLaunchKernelEx(&cfg, mla_decode_kernel<false>, prm);
 }
 
 }  // namespace mla

@@ -28,7 +28,6 @@
 namespace mla {
 namespace {
 
-constexpr int kRowBytes = 656;
 constexpr int kWarpsPerBlock = 8;
 
 // two fp32 -> two e4m3 (round to nearest even, saturating), lo in the low byte
@@ -44,7 +43,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) quantize_kernel(const __n
   const int64_t row = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   if (row >= rows) return;
   const __nv_bfloat16* src = kv + row * kDQK;
-  uint8_t* dst = out + row * kRowBytes;
+  uint8_t* dst = out + row * kRowBytes8;
   // c_kv[16 lane .. 16 lane + 15]
   const uint4 a = reinterpret_cast<const uint4*>(src)[2 * lane];
   const uint4 b = reinterpret_cast<const uint4*>(src)[2 * lane + 1];
@@ -92,9 +91,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) quantize_kernel(const __n
   reinterpret_cast<uint4*>(dst)[lane] = make_uint4(q[0], q[1], q[2], q[3]);
   // scaled k_pe (128 bytes) by lanes 0-7, then the scale and the zero pad by lane 8
   if (lane < 8) {
-    reinterpret_cast<uint4*>(dst + 512)[lane] = make_uint4(kq[0], kq[1], kq[2], kq[3]);
+    reinterpret_cast<uint4*>(dst + kOffKpe8)[lane] = make_uint4(kq[0], kq[1], kq[2], kq[3]);
   } else if (lane == 8) {
-    reinterpret_cast<uint4*>(dst + 640)[0] = make_uint4(__float_as_uint(scale), 0u, 0u, 0u);
+    reinterpret_cast<uint4*>(dst + kOffScale8)[0] = make_uint4(__float_as_uint(scale), 0u, 0u, 0u);
   }
 }
 

@@ -13,6 +13,12 @@ constexpr int kRowsPerCta = 64;    // each CTA of the pair owns 64 of them
 constexpr int kTileKeys = 256;     // keys per pipeline step (4 cache blocks)
 constexpr int kBlocksPerTile = kTileKeys / kBlockSize;
 
+// Packed FP8 cache row (bytes): [0, 512) e4m3 codes of c_kv / scale, [512, 640) k_pe /
+// scale as 64 bf16, [640, 644) the fp32 scale, [644, 656) zero.
+constexpr int kRowBytes8 = 656;
+constexpr int kOffKpe8 = 512;
+constexpr int kOffScale8 = 640;
+
 // Split-KV scheduler constants (the same values are stated in the float64 oracle).
 constexpr int kSchedOverheadTiles = 1;  // cost of starting a sequence, in 256-key tiles
 constexpr int kSchedMinCap = 2;         // smallest partition cost, in tiles

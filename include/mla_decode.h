@@ -279,6 +279,31 @@ mla_status_t mla_absorb_out(const void* o_latent, const void* w_uv, void* y, int
  */
 mla_status_t mla_quantize_kv_fp8(const void* kv_cache, void* kv_fp8, int64_t rows, void* stream);
 
+/*
+ * mla_decode_fp8: mla_decode_ragged over a packed FP8 cache (the format above): the
+ * same arguments, with `kv_fp8` = [num_blocks][64][656] bytes (device, 16-byte aligned)
+ * in place of the bf16 cache; q_lens may be NULL (s_q tokens for every sequence).  The
+ * result is the decode of the dequantised rows scale * [e4m3(code) | k_pe'] (the FP8
+ * cache is 8-bit KV-cache inference, Paddle 3.0 inference upgrade article, closing
+ * capabilities list).  The schedule, workspace, error statuses and asynchrony are
+ * those of mla_decode.
+ */
+mla_status_t mla_decode_fp8(const void* q_nope, const void* q_pe, const void* kv_fp8, int64_t num_blocks,
+                            const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                            const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
+                            const void* metadata, size_t metadata_bytes, void* workspace, size_t workspace_bytes,
+                            void* out, float* lse, int32_t* status, void* stream);
+
+/* mla_decode_fp8_attention: the split-KV attention launch of mla_decode_fp8 alone (its
+ * LSE combine is mla_decode_combine, as for mla_decode_attention).  Same arguments and
+ * passage as mla_decode_fp8; used to time the attention kernel by itself. */
+mla_status_t mla_decode_fp8_attention(const void* q_nope, const void* q_pe, const void* kv_fp8, int64_t num_blocks,
+                                      const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                                      const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
+                                      const void* metadata, size_t metadata_bytes, void* workspace,
+                                      size_t workspace_bytes, void* out, float* lse, int32_t* status,
+                                      void* stream);
+
 /* Number of streaming multiprocessors the schedule targets on the current device.
  * Library convenience: no passage of the source pages corresponds to it. */
 mla_status_t mla_device_sm_count(int* sm_count);

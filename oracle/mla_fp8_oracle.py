@@ -151,8 +151,10 @@ def dequantize_cache(packed: np.ndarray) -> np.ndarray:
     return np.concatenate([e4m3_decode(codes) * s, O.bf16_to_f64(kpe) * s], axis=-1)
 
 
-def mla_decode_fp8_ref(q_nope, q_pe, kv_fp8_packed, block_table, cache_seqlens, softmax_scale, causal):
+def mla_decode_fp8_ref(q_nope, q_pe, kv_fp8_packed, block_table, cache_seqlens, softmax_scale, causal,
+                       q_lens=None):
     """Decode over the packed FP8 cache: the float64 definition of ``mla_decode_ref``
-    applied to the dequantised rows (q_nope / q_pe float64 as there)."""
+    applied to the dequantised rows (q_nope / q_pe float64 as there; q_lens, the
+    per-sequence query counts, as there)."""
     return O.mla_decode_ref(q_nope, q_pe, dequantize_cache(kv_fp8_packed), block_table, cache_seqlens,
-                            softmax_scale, causal)
+                            softmax_scale, causal, q_lens=q_lens)

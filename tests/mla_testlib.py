@@ -6,6 +6,7 @@ from __future__ import annotations
 import numpy as np
 
 from oracle import mla_oracle as O
+from oracle import mla_fp8_oracle as F
 
 # Tolerances against the float64 oracle (the acceptance bar of this library):
 # out max-abs <= 2e-2 and mean-abs <= 2e-3, lse max-abs <= 1e-3.
@@ -60,6 +61,43 @@ def oracle(inp, seqs=None, q_lens=None):
         o, l = O.mla_decode_ref(qn[b : b + 1], qp[b : b + 1], kv_b if nblk else np.zeros((1, 64, 576)), table,
                                 np.array([n]), inp.softmax_scale, inp.causal,
                                 q_lens=None if q_lens is None else np.asarray(q_lens)[b : b + 1])
+        outs.append(o[0])
+        lses.append(l[0])
+    return np.stack(outs), np.stack(lses)
+
+
+def run_cuda_fp8(inp, dev=None, status=None, q_lens=None):
+    """The FP8 path: mla_quantize_kv_fp8 of the bf16 cache, then mla_get_metadata +
+    mla_decode_fp8; returns (out f64, lse f64, meta)."""
+    import torch
+    import deepseek_mla_decode_b200 as mla
+
+    dev = dev or to_device(inp)
+    kv8 = mla.quantize_kv_fp8(dev["kv_cache"])
+    meta = mla.get_metadata(dev["cache_seqlens"], inp.s_q, inp.H)
+    ql = None if q_lens is None else torch.tensor(np.asarray(q_lens, dtype=np.int32)).cuda()
+    out, lse = mla.decode_fp8(dev["q_nope"], dev["q_pe"], kv8, dev["block_table"], dev["cache_seqlens"],
+                              inp.softmax_scale, inp.causal, meta, q_lens=ql, status=status)
+    torch.cuda.synchronize()
+    return out.float().cpu().double().numpy(), lse.cpu().double().numpy(), meta
+
+
+def oracle_fp8(inp, seqs=None, q_lens=None):
+    """FP8 oracle: the oracle's own quantiser packs the bf16 cache, then the decode
+    over the dequantised rows; per sequence (its blocks only) when seqs is given."""
+    qn, qp = O.bf16_to_f64(inp.q_nope), O.bf16_to_f64(inp.q_pe)
+    if seqs is None:
+        return F.mla_decode_fp8_ref(qn, qp, F.pack_cache(inp.kv_cache), inp.block_table, inp.cache_seqlens,
+                                    inp.softmax_scale, inp.causal, q_lens=q_lens)
+    outs, lses = [], []
+    for b in seqs:
+        n = int(inp.cache_seqlens[b])
+        nblk = (n + 63) // 64
+        ids = inp.block_table[b, :nblk]
+        packed = F.pack_cache(inp.kv_cache[ids]) if nblk else np.zeros((1, 64, F.ROW_BYTES), np.uint8)
+        table = np.arange(max(nblk, 1))[None, :]
+        o, l = F.mla_decode_fp8_ref(qn[b : b + 1], qp[b : b + 1], packed, table, np.array([n]), inp.softmax_scale,
+                                    inp.causal, q_lens=None if q_lens is None else np.asarray(q_lens)[b : b + 1])
         outs.append(o[0])
         lses.append(l[0])
     return np.stack(outs), np.stack(lses)
