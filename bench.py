@@ -326,9 +326,11 @@ class DeviceRun:
         import torch
 
         i, m, st = self.inp, self.mla, self.stream
+        # the cache as the caller holds it: bf16 rows, or the packed FP8 rows
+        kv_host = self.kv.cpu().numpy() if self.fp8 else i.kv_cache.view(np.int16)
         h = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for k, v in
              (("q_nope", i.q_nope.view(np.int16)), ("q_pe", i.q_pe.view(np.int16)),
-              ("kv", i.kv_cache.view(np.int16)), ("table", i.block_table), ("seq", i.cache_seqlens))}
+              ("kv", kv_host), ("table", i.block_table), ("seq", i.cache_seqlens))}
         h_out = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
         h_lse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
         d = {k: torch.empty(v.shape, dtype=v.dtype, device=self.dev) for k, v in h.items()}
@@ -339,9 +341,14 @@ class DeviceRun:
             for k in h:
                 d[k].copy_(h[k], non_blocking=True)
             meta = m.get_metadata(d["seq"], i.s_q, i.H, metadata=self.meta, stream=st)
-            m.decode(d["q_nope"].view(torch.bfloat16), d["q_pe"].view(torch.bfloat16), d["kv"].view(torch.bfloat16),
-                     d["table"], d["seq"], i.softmax_scale, i.causal, meta, workspace=self.ws, out=self.out,
-                     lse=self.lse, status=self.status, stream=st)
+            if self.fp8:
+                m.decode_fp8(d["q_nope"].view(torch.bfloat16), d["q_pe"].view(torch.bfloat16), d["kv"], d["table"],
+                             d["seq"], i.softmax_scale, i.causal, meta, workspace=self.ws, out=self.out,
+                             lse=self.lse, status=self.status, stream=st)
+            else:
+                m.decode(d["q_nope"].view(torch.bfloat16), d["q_pe"].view(torch.bfloat16), d["kv"].view(torch.bfloat16),
+                         d["table"], d["seq"], i.softmax_scale, i.causal, meta, workspace=self.ws, out=self.out,
+                         lse=self.lse, status=self.status, stream=st)
             h_out.copy_(self.out, non_blocking=True)
             h_lse.copy_(self.lse, non_blocking=True)
 
@@ -399,6 +406,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="serving_b256", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--kv-format", default="bf16", choices=["bf16", "fp8"],
+                    help="cache of the headline run: bf16 rows, or the packed FP8 rows (quantised once, untimed)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -458,7 +467,10 @@ def main():
     inp = make_workload(args.workload)
     flops, cache_bytes, algo_bytes = algorithmic_work(inp.cache_seqlens, inp.s_q, inp.H, inp.causal)
     B, s_q, H = inp.B, inp.s_q, inp.H
-    run = DeviceRun(mla, inp, dev)
+    fp8 = args.kv_format == "fp8"
+    if fp8:
+        flops, cache_bytes, algo_bytes = algorithmic_work(inp.cache_seqlens, inp.s_q, inp.H, inp.causal, 656)
+    run = DeviceRun(mla, inp, dev, fp8=fp8)
 
     run.steps(args.warmup, flusher)
     torch.cuda.synchronize()
@@ -505,7 +517,7 @@ def main():
         del run
         torch.cuda.empty_cache()
         for name in ("decode_b64", "mtp_b128_sq2", "serving_b256", "long_b4"):
-            if name == args.workload:
+            if name == args.workload and not fp8:
                 continue
             wi = make_workload(name)
             ri = DeviceRun(mla, wi, dev)
@@ -518,6 +530,8 @@ def main():
             torch.cuda.empty_cache()
         # the four full-size decode configurations over the packed FP8 cache (656-byte rows)
         for name in ("serving_b256", "decode_b64", "mtp_b128_sq2", "long_b4"):
+            if name == args.workload and fp8:
+                continue
             wi = make_workload(name)
             ri = DeviceRun(mla, wi, dev, fp8=True)
             ri.steps(args.warmup, flusher)
@@ -535,13 +549,15 @@ def main():
 
     ms = step_ms / K
     value = whole_job_rate(world, flops, ms) / 1e12
-    roof = roofline(inp, {"attention": att_ms, "step": step_ser_ms, "metadata": meta_ms, "combine": comb_ms}, K)
-    per_workload[w.name] = {k: roof[k] for k in ("bound", "kernel_avg_us", "roofline_us", "pct_of_roofline", "frac",
-                                                 "step_us", "step_without_metadata_us", "pct_of_roofline_decode")}
-    roof["traffic"] = recorded_traffic(w.name)
+    roof = roofline(inp, {"attention": att_ms, "step": step_ser_ms, "metadata": meta_ms, "combine": comb_ms}, K,
+                    fp8=fp8)
+    per_workload[w.name + ("_fp8" if fp8 else "")] = {
+        k: roof[k] for k in ("bound", "kernel_avg_us", "roofline_us", "pct_of_roofline", "frac", "step_us",
+                             "step_without_metadata_us", "pct_of_roofline_decode")}
+    roof["traffic"] = recorded_traffic(w.name + ("_fp8" if fp8 else ""))
 
     line = {
-        "metric": metric_name(w),
+        "metric": metric_name(w) + (" [FP8 cache]" if fp8 else ""),
         "value": value,
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -551,9 +567,10 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16" if not fp8 else "bf16 (e4m3 cache)",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": B, "s_q": s_q, "H": H, "causal": w.causal, "lengths": w.lengths,
+        "config": {"workload": w.name, "kv_format": args.kv_format, "B": B, "s_q": s_q, "H": H, "causal": w.causal,
+                   "lengths": w.lengths,
                    "seed": w.seed, "block_size": 64, "softmax_scale": inp.softmax_scale,
                    "l2": L2Flush.DESCRIPTION,
                    "parallelism": f"replicas x{world}"},
