@@ -42,6 +42,10 @@ EXPORTED_SYMBOLS = (
     "mla_quantize_kv_fp8",
     "mla_decode_fp8",
     "mla_decode_fp8_attention",
+    "mla_sage_workspace_size",
+    "mla_sage_quantize",
+    "mla_sage_attention",
+    "mla_sage_prefill",
 )
 
 _lib = None
@@ -95,6 +99,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         fn.argtypes = [c_vp, c_vp, c_vp, c_int, c_int, c_vp]
     L.mla_quantize_kv_fp8.restype = c_int
     L.mla_quantize_kv_fp8.argtypes = [c_vp, c_vp, c_i64, c_vp]
+    L.mla_sage_workspace_size.restype = c_int
+    L.mla_sage_workspace_size.argtypes = [c_int, c_int, ctypes.POINTER(c_size)]
+    L.mla_sage_quantize.restype = c_int
+    L.mla_sage_quantize.argtypes = [c_vp, c_vp, c_vp, c_int, c_int, c_vp, c_size, c_vp]
+    L.mla_sage_attention.restype = c_int
+    L.mla_sage_attention.argtypes = [c_int, c_int, c_f, c_vp, c_size, c_vp, c_vp, c_vp, c_vp]
+    L.mla_sage_prefill.restype = c_int
+    L.mla_sage_prefill.argtypes = [c_vp, c_vp, c_vp, c_int, c_int, c_f, c_vp, c_size, c_vp, c_vp, c_vp, c_vp]
     L.mla_decode_noalloc.restype = c_int
     L.mla_decode_noalloc.argtypes = [c_vp, c_vp, c_vp, c_i64, c_vp, c_int, c_vp, c_int, c_int, c_int, c_f, c_int,
                                      c_vp, c_size, c_vp, c_vp, c_vp, c_vp]
@@ -238,6 +250,67 @@ def decode_fp8_attention(q_nope, q_pe, kv_fp8, block_table, cache_seqlens, softm
                         workspace, out, lse, status, stream)
     _check("mla_decode_fp8_attention", load_library().mla_decode_fp8_attention(
         *args[:7], q_lens.data_ptr() if q_lens is not None else None, *args[7:]))
+
+
+def sage_workspace_size(S: int, H: int) -> int:
+    n = ctypes.c_size_t()
+    _check("mla_sage_workspace_size", load_library().mla_sage_workspace_size(S, H, ctypes.byref(n)))
+    return n.value
+
+
+def _sage_check(q, k, v):
+    S, H, dq = q.shape
+    if dq != 192 or tuple(k.shape) != (S, H, 192) or tuple(v.shape) != (S, H, 128):
+        raise ValueError("q, k [S, H, 192] and v [S, H, 128] expected")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    return S, H
+
+
+def sage_quantize(q, k, v, workspace=None, stream=None):
+    """mla_sage_quantize: the INT8 / FP8 codes and scales of q, k, v in a workspace
+    (uint8 tensor; layout in include/mla_decode.h)."""
+    import torch
+
+    S, H = _sage_check(q, k, v)
+    if workspace is None:
+        workspace = torch.empty(sage_workspace_size(S, H), dtype=torch.uint8, device=q.device)
+    _check("mla_sage_quantize", load_library().mla_sage_quantize(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), S, H, workspace.data_ptr(), workspace.numel(), _stream_ptr(stream)))
+    return workspace
+
+
+def sage_attention(S: int, H: int, softmax_scale: float, workspace, out=None, lse=None, status=None, stream=None):
+    """mla_sage_attention over a filled workspace; returns (out bf16 [S, H, 128], lse fp32 [S, H])."""
+    import torch
+
+    if out is None:
+        out = torch.empty((S, H, 128), dtype=torch.bfloat16, device=workspace.device)
+    if lse is None:
+        lse = torch.empty((S, H), dtype=torch.float32, device=workspace.device)
+    _check("mla_sage_attention", load_library().mla_sage_attention(
+        S, H, float(softmax_scale), workspace.data_ptr(), workspace.numel(), out.data_ptr(), lse.data_ptr(),
+        status.data_ptr() if status is not None else None, _stream_ptr(stream)))
+    return out, lse
+
+
+def sage_prefill(q, k, v, softmax_scale: float, workspace=None, out=None, lse=None, status=None, stream=None):
+    """mla_sage_prefill: quantised causal prefill attention (q, k [S, H, 192], v [S, H, 128],
+    bf16); returns (out bf16 [S, H, 128], lse fp32 [S, H])."""
+    import torch
+
+    S, H = _sage_check(q, k, v)
+    if workspace is None:
+        workspace = torch.empty(sage_workspace_size(S, H), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((S, H, 128), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((S, H), dtype=torch.float32, device=q.device)
+    _check("mla_sage_prefill", load_library().mla_sage_prefill(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), S, H, float(softmax_scale), workspace.data_ptr(), workspace.numel(),
+        out.data_ptr(), lse.data_ptr(), status.data_ptr() if status is not None else None, _stream_ptr(stream)))
+    return out, lse
 
 
 def absorb_q(q_heads, w_uk, q_nope=None, stream=None):

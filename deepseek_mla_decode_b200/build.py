@@ -19,8 +19,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmla.so")
 SOURCES = ["mla_api.cu", "mla_metadata.cu", "mla_decode_kernel.cu", "mla_combine.cu", "mla_noalloc.cu",
-           "mla_absorb.cu", "mla_fp8.cu"]
-HEADERS = ["mla_internal.h", "ptx_sm100.cuh"]
+           "mla_absorb.cu", "mla_fp8.cu", "sage_quant.cu", "sage_attn.cu"]
+HEADERS = ["mla_internal.h", "ptx_sm100.cuh", "sage_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

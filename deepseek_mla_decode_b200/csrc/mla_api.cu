@@ -8,6 +8,7 @@
 #include <atomic>
 #include <mutex>
 #include "mla_internal.h"
+#include "sage_internal.h"
 #include "../../include/mla_decode.h"
 
 namespace mla {
@@ -17,6 +18,12 @@ cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, const in
                            int B, int s_q, int M, int P, const float* part_o, const float* part_lse, void* out,
                            float* lse, cudaStream_t stream);
 cudaError_t decode_kernel_setup(int device);
+namespace sage {
+cudaError_t attention_setup();
+cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                             const Workspace& ws, int S, int H, float softmax_scale, void* out, float* lse,
+                             int32_t* status, uint64_t timeout_ns, cudaStream_t stream);
+}  // namespace sage
 cudaError_t launch_decode(bool fp8, const CUtensorMap& tm_kv, const CUtensorMap& tm_kv2,
                           const CUtensorMap* tm_kpe, const CUtensorMap* tm_scl,
                           const CUtensorMap& tm_qn, const CUtensorMap& tm_qp,
@@ -65,6 +72,7 @@ mla_status_t device_info(int* sm_count) {
       return MLA_ERR_CUDA;
     if (major != 10 || minor != 0) return MLA_ERR_DEVICE;
     if (mla::decode_kernel_setup(dev) != cudaSuccess) return MLA_ERR_CUDA;
+    if (mla::sage::attention_setup() != cudaSuccess) return MLA_ERR_CUDA;
     if (!g_encode) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -447,6 +455,79 @@ mla_status_t mla_decode_fp8_attention(const void* q_nope, const void* q_pe, cons
   return launch_attention(true, q_nope, q_pe, kv_fp8, num_blocks, block_table, max_blocks, cache_seqlens, q_lens,
                           B, s_q, H, softmax_scale, causal, metadata, workspace, out, lse, status, g,
                           static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// quantised prefill attention (SageAttention-style, head dim 192)
+// ---------------------------------------------------------------------------
+mla_status_t mla_sage_workspace_size(int S, int H, size_t* bytes) {
+  if (!bytes || S < 1 || H < 1 || H > 65535) return MLA_ERR_INVALID_ARG;
+  if ((int64_t)mla::sage::padded_len(S) / mla::sage::kBlockM * H > 0x7fffffffLL) return MLA_ERR_UNSUPPORTED;
+  *bytes = mla::sage::workspace_bytes(S, H);
+  return MLA_OK;
+}
+
+mla_status_t mla_sage_quantize(const void* q, const void* k, const void* v, int S, int H, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !workspace) return MLA_ERR_INVALID_ARG;
+  size_t need = 0;
+  mla_status_t st = mla_sage_workspace_size(S, H, &need);
+  if (st != MLA_OK) return st;
+  if (workspace_bytes < need) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
+  int sms = 0;
+  st = device_info(&sms);
+  if (st != MLA_OK) return st;
+  const mla::sage::Workspace ws = mla::sage::carve(workspace, S, H);
+  if (mla::sage::launch_quantize(q, k, v, S, H, ws, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+mla_status_t mla_sage_attention(int S, int H, float softmax_scale, const void* workspace, size_t workspace_bytes,
+                                void* out, float* lse, int32_t* status, void* stream) {
+  if (!workspace || !out || !lse) return MLA_ERR_INVALID_ARG;
+  size_t need = 0;
+  mla_status_t st = mla_sage_workspace_size(S, H, &need);
+  if (st != MLA_OK) return st;
+  if (workspace_bytes < need) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (!(softmax_scale > 0.f) || softmax_scale > 1e30f) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(workspace) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(status) & 3u))
+    return MLA_ERR_INVALID_ARG;
+  int sms = 0;
+  st = device_info(&sms);
+  if (st != MLA_OK) return st;
+  const mla::sage::Workspace ws = mla::sage::carve(const_cast<void*>(workspace), S, H);
+  const int S_pad = mla::sage::padded_len(S);
+  CUtensorMap tm_q, tm_k, tm_v;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)mla::sage::kDQK, (cuuint64_t)S_pad, (cuuint64_t)H};
+    cuuint64_t strides[2] = {(cuuint64_t)mla::sage::kDQK, (cuuint64_t)mla::sage::kDQK * S_pad};
+    cuuint32_t box[3] = {64, (cuuint32_t)mla::sage::kBlockM, 1};
+    if (!encode(&tm_q, ws.q8, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode(&tm_k, ws.k8, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_64B))
+      return MLA_ERR_INVALID_ARG;
+  }
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)S_pad, (cuuint64_t)mla::sage::kDV * H};
+    cuuint64_t strides[1] = {(cuuint64_t)S_pad};
+    cuuint32_t box[2] = {(cuuint32_t)mla::sage::kBlockN, (cuuint32_t)mla::sage::kDV};
+    if (!encode(&tm_v, ws.vt8, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_INVALID_ARG;
+  }
+  if (mla::sage::launch_attention(tm_q, tm_k, tm_v, ws, S, H, softmax_scale, out, lse, status,
+                                  g_wait_timeout_ns.load(), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+mla_status_t mla_sage_prefill(const void* q, const void* k, const void* v, int S, int H, float softmax_scale,
+                              void* workspace, size_t workspace_bytes, void* out, float* lse, int32_t* status,
+                              void* stream) {
+  mla_status_t st = mla_sage_quantize(q, k, v, S, H, workspace, workspace_bytes, stream);
+  if (st != MLA_OK) return st;
+  return mla_sage_attention(S, H, softmax_scale, workspace, workspace_bytes, out, lse, status, stream);
 }
 
 }  // extern "C"

@@ -304,6 +304,42 @@ mla_status_t mla_decode_fp8_attention(const void* q_nope, const void* q_pe, cons
                                       size_t workspace_bytes, void* out, float* lse, int32_t* status,
                                       void* stream);
 
+/*
+ * Quantised causal prefill attention, head dimension 192 (SageAttention-style: Paddle
+ * 3.0 inference upgrade article, long-sequence section -- Q and K dynamically
+ * quantised to INT8 and V to FP8, the INT32 scores converted to FP32 and dequantised,
+ * an online softmax, P quantised to FP8 and multiplied with the FP8 V, the product
+ * dequantised by V's scale; DeepSeek's head dimension 192).
+ *
+ * Inputs (device, 16-byte aligned, bf16, row-major): q, k [S][H][192] (query i is
+ * token i of one sequence; key j is visible to query i when j <= i), v [S][H][128].
+ * Outputs: out [S][H][128] bf16, lse [S][H] fp32 (natural log of the sum of the
+ * quantised weights, scale included).  Quantisation (this library's reading of the
+ * passage): Q and K per (token, head), scale = max|x| / 127, code = rint(x / scale);
+ * V per (head, channel) over all tokens, scale = max|v| / 448, code = e4m3(v / scale);
+ * P = 2^(x - m) in [0, 1] at the running row maximum m of 128-key blocks, coded as
+ * e4m3(P * 448); the output is normalised by the sum of the coded weights.
+ *
+ * mla_sage_workspace_size: bytes of the workspace for (S, H): the codes and scales,
+ *   S_pad = S rounded up to 128: q8, k8 int8 [H][S_pad][192]; vt8 e4m3 [H][128][S_pad]
+ *   (V transposed); sq, sk fp32 [H][S_pad]; sv fp32 [H][128]; uint32 [H][128] scratch.
+ *   1 <= S, 1 <= H <= 65535.
+ * mla_sage_quantize: fill the workspace from q, k, v (asynchronous on `stream`).
+ * mla_sage_attention: the attention kernel over a filled workspace.  status (device
+ *   int32, may be NULL) gets MLA_DEVICE_ERR_TIMEOUT if a pipeline wait ran out.
+ * mla_sage_prefill: mla_sage_quantize then mla_sage_attention.
+ * Host-detectable errors return before any launch; the workspace belongs to the caller
+ * and must not be shared by concurrent calls.
+ */
+mla_status_t mla_sage_workspace_size(int S, int H, size_t* bytes);
+mla_status_t mla_sage_quantize(const void* q, const void* k, const void* v, int S, int H, void* workspace,
+                               size_t workspace_bytes, void* stream);
+mla_status_t mla_sage_attention(int S, int H, float softmax_scale, const void* workspace, size_t workspace_bytes,
+                                void* out, float* lse, int32_t* status, void* stream);
+mla_status_t mla_sage_prefill(const void* q, const void* k, const void* v, int S, int H, float softmax_scale,
+                              void* workspace, size_t workspace_bytes, void* out, float* lse, int32_t* status,
+                              void* stream);
+
 /* Number of streaming multiprocessors the schedule targets on the current device.
  * Library convenience: no passage of the source pages corresponds to it. */
 mla_status_t mla_device_sm_count(int* sm_count);
