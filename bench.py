@@ -63,6 +63,58 @@ def algorithmic_work(seqlens, s_q, H, causal, row_bytes=D_QK * 2):
     return flops, cache_bytes, cache_bytes + q_bytes + out_bytes
 
 
+def prefill_work(S, H):
+    """Operations of the causal quantised prefill: 2 (192 + 128) per (head, query,
+    visible key), S (S + 1) / 2 visible pairs per head."""
+    return 2.0 * (192 + 128) * H * S * (S + 1) / 2
+
+
+def bench_prefill(mla, dev, steps, warmup):
+    """Quantised causal prefill (64K tokens, 16 heads, head dim 192) on seeded device
+    inputs (N(0, 1) bf16 from a seeded torch generator; the inputs and the quantised
+    workspace exceed L2).  Returns the per-workload entry: quantiser and attention
+    kernel times (CUDA events) and the attention kernel's tensor roofline against the
+    8-bit dense peak (twice the bf16 peak)."""
+    import torch
+    from deepseek_mla_decode_b200.workloads import PREFILL_S, PREFILL_H, PREFILL_SEED
+
+    S, H = PREFILL_S, PREFILL_H
+    g = torch.Generator(device=dev).manual_seed(PREFILL_SEED)
+    q = torch.randn((S, H, 192), generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn((S, H, 192), generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn((S, H, 128), generator=g, device=dev).to(torch.bfloat16)
+    ws = torch.empty(mla.sage_workspace_size(S, H), dtype=torch.uint8, device=dev)
+    out = torch.empty((S, H, 128), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((S, H), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    st = torch.cuda.current_stream()
+    scale = 1.0 / math.sqrt(192.0)
+    for _ in range(warmup):
+        mla.sage_prefill(q, k, v, scale, workspace=ws, out=out, lse=lse, status=status, stream=st)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for e in ev:
+        e[0].record(st)
+        mla.sage_quantize(q, k, v, workspace=ws, stream=st)
+        e[1].record(st)
+        mla.sage_attention(S, H, scale, ws, out=out, lse=lse, status=status, stream=st)
+        e[2].record(st)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} in the prefill")
+    quant_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+    att_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+    _, bf16_peak, _, src = load_peaks()
+    peak = 2 * bf16_peak
+    ops = prefill_work(S, H)
+    achieved = ops / (att_ms * 1e-3) / 1e12
+    return {"workload": f"causal prefill S={S}, H={H}, head dim 192 / 128", "kernel": "sage_attn_kernel",
+            "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_source": f"{src} bf16 GEMM x 2 (dense 8-bit)", "kernel_avg_us": att_ms * 1e3,
+            "roofline_us": ops / (peak * 1e12) * 1e6, "quantize_us": quant_ms * 1e3,
+            "tokens_per_s": S / ((att_ms + quant_ms) * 1e-3), "steps": steps}
+
+
 def metric_name(w):
     """The metric string both arms print, so their lines can be divided."""
     return f"MLA decode TFLOP/s ({w.name}: B={w.B}, s_q={w.s_q}, H={w.H})"
@@ -406,6 +458,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="serving_b256", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--prefill-steps", type=int, default=5,
+                    help="timed runs of the quantised 64K-token prefill (0 = skip)")
     ap.add_argument("--kv-format", default="bf16", choices=["bf16", "fp8"],
                     help="cache of the headline run: bf16 rows, or the packed FP8 rows (quantised once, untimed)")
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -541,6 +595,10 @@ def main():
             per_workload[name + "_fp8"] = roofline(wi, ti, args.per_workload_steps, fp8=True)
             del ri
             torch.cuda.empty_cache()
+
+    if world == 1 and args.prefill_steps > 0:
+        per_workload["prefill_s65536_h16"] = bench_prefill(mla, dev, args.prefill_steps, 2)
+        torch.cuda.empty_cache()
 
     if rank != 0:
         if world > 1:

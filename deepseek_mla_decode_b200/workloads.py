@@ -175,3 +175,21 @@ def make_up_projections(H: int, seed: int, scale: float = 0.05):
 def make_rows(shape, seed: int):
     """bf16 bit patterns of N(0, 1) draws with the given shape."""
     return _normal_bf16(np.random.default_rng(seed), shape)
+
+
+# ---------------------------------------------------------------------------
+# quantised prefill (SageAttention-style, head dim 192)
+# ---------------------------------------------------------------------------
+# The long-prompt prefill of the Paddle 3.0 inference article's long-sequence section:
+# a 64K-token prompt with DeepSeek's head dimension 192 (V 128).  16 heads is one GPU's
+# share of the 128 query heads under 8-way tensor parallelism.
+PREFILL_S, PREFILL_H, PREFILL_SEED = 65536, 16, 2024
+
+
+def make_prefill(S: int, H: int, seed: int):
+    """q, k as bf16 bits [S, H, 192] and v [S, H, 128], N(0, 1)."""
+    rng = np.random.default_rng(seed)
+    q = _normal_bf16(rng, (S, H, 192))
+    k = _normal_bf16(rng, (S, H, 192))
+    v = _normal_bf16(rng, (S, H, 128))
+    return q, k, v
