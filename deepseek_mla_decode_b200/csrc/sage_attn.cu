@@ -16,7 +16,9 @@
 // One CTA = one head x 128 query rows.  Warp 0 issues the TMA loads (Q once; per key
 // block its K slab, V slab and the keys' scales), warp 1 the MMAs (QK of block j+1 is
 // issued before PV of block j, so the tensor core works while the softmax runs),
-// warps 4..7 the softmax (one thread per query row = TMEM lane) and the epilogue.
+// warps 4..11 the softmax and the epilogue (two threads per query row: warps 4..7 take
+// keys / output columns 0..63 of each block, warps 8..11 columns 64..127; a row's TMEM
+// lane is reachable from both, lane quadrant = warp % 4).
 // TMEM: S double buffer in columns [0, 256), O in [256, 384).  Every wait is bounded:
 // a timeout sets MLA_DEVICE_ERR_TIMEOUT, every role stops at its next wait, the CTA
 // drains its tensor-core work and returns.
@@ -36,8 +38,9 @@ using namespace ptx;
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kProducerWarp = 0, kMmaWarp = 1, kSoftmaxWarp0 = 4;
+constexpr int kSoftmaxThreads = 256;  // warps 4..11: two threads per query row, 64 keys each
 constexpr int kStages = 4;
 constexpr int kChunk = kBlockN * 64;          // one [128 rows][64 B] SW64 box (8 KB)
 constexpr int kQBytes = 3 * kChunk;           // Q: 128 rows x 192 B
@@ -81,12 +84,14 @@ struct __align__(8) Ctrl {
   uint64_t empty[kStages];  // PV of the stage's block done (commit)
   uint64_t q_full;
   uint64_t s_full[2];       // S buffer written (commit)
-  uint64_t s_free[2];       // S buffer read by the 128 softmax threads
+  uint64_t s_free[2];       // S buffer read by the 256 softmax threads
   uint64_t p_full;          // P written and O rescaled (one arrive)
   uint64_t p_free;          // PV done (commit)
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort;
+  float red_max[2][2][kBlockM];  // per block parity, column half, row: block maximum
+  float red_l[2][kBlockM];       // per column half, row: sum of coded weights
 };
 
 __device__ __forceinline__ void set_status(const Params& p, int bits) {
@@ -169,15 +174,16 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
 }
-// sum of the values of the two e4m3 codes in the low 16 bits of c
-__device__ __forceinline__ float e4m3x2_sum(uint32_t c) {
-  uint32_t h2;
-  asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(h2) : "r"(c));
-  float a, b;
-  asm("{\n\t.reg .b16 x, y;\n\tmov.b32 {x, y}, %2;\n\tcvt.f32.f16 %0, x;\n\tcvt.f32.f16 %1, y;\n\t}"
-      : "=f"(a), "=f"(b)
-      : "r"(h2));
-  return a + b;
+// acc + the values of the two e4m3 codes in the low 16 bits of c (exact f16 values,
+// added to the fp32 accumulator by the mixed-precision f32 += f16 add)
+__device__ __forceinline__ float add_e4m3x2_to(float acc, uint32_t c) {
+  float r;
+  asm("{\n\t.reg .b16 lo, x, y;\n\t.reg .b32 h2;\n\t.reg .f32 t;\n\tcvt.u16.u32 lo, %1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h2, lo;\n\tmov.b32 {x, y}, h2;\n\t"
+      "add.rn.f32.f16 t, x, %2;\n\tadd.rn.f32.f16 %0, y, t;\n\t}"
+      : "=f"(r)
+      : "r"(c), "f"(acc));
+  return r;
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
@@ -210,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
     mbar_init(smem_u32(&ctrl.q_full), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&ctrl.s_full[s]), 1);
-      mbar_init(smem_u32(&ctrl.s_free[s]), kBlockM);
+      mbar_init(smem_u32(&ctrl.s_free[s]), kSoftmaxThreads);
     }
     mbar_init(smem_u32(&ctrl.p_full), 1);
     mbar_init(smem_u32(&ctrl.p_free), 1);
@@ -309,9 +315,10 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
     }
   } else if (warp >= kSoftmaxWarp0) {
     // =====================================================================
-    // softmax + epilogue: thread = query row r = TMEM lane r
+    // softmax + epilogue: thread (g, r) = query row r (TMEM lane r), columns 64g..64g+63
     // =====================================================================
-    const int r = tid - kSoftmaxWarp0 * 32;
+    const int st = tid - kSoftmaxWarp0 * 32;  // 0..255
+    const int g = st >> 7, r = st & 127;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const int row = qb * kBlockM + r;
     const bool valid = row < p.S;
@@ -320,45 +327,66 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
     bool ok = true, go = true;
     const float* sc_all = reinterpret_cast<const float*>(smem + kSmemScale);
     for (int j = 0; j < nkb && go; ++j) {
-      const int st = j % kStages;
+      const int stg = j % kStages;
       ok = wait_bar(&ctrl, p, smem_u32(&ctrl.s_full[j & 1]), (j >> 1) & 1) && ok;
       // the stage's scales landed with its TMA (already complete; this wait makes them
       // visible to these threads)
-      ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[st]), (j / kStages) & 1) && ok;
+      ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[stg]), (j / kStages) & 1) && ok;
       tc_fence_after();
-      uint32_t s[128];
+      uint32_t s[64];
       if (ok) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          tmem_ld32(tmem + kTmemS0 + 128 * (j & 1) + lane_off + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
+        const uint32_t ta = tmem + kTmemS0 + 128 * (j & 1) + lane_off + 64 * g;
+        tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
         tmem_wait_ld();
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&ctrl.s_free[j & 1]));  // the S buffer may be overwritten
-      // dequantised log2-scaled scores of the visible keys (key j*128 + c <= row)
-      const float* sc = sc_all + st * kBlockN;
-      const int vis = valid ? min(kBlockN, row - j * kBlockN + 1) : 0;
-      float bmax = -INFINITY;
+      // dequantised log2-scaled scores of the visible keys (key j*128 + 64g + c <= row)
+      const float* sc = sc_all + stg * kBlockN + 64 * g;
+      const int vis = valid ? max(0, min(64, row - j * kBlockN - 64 * g + 1)) : 0;
+      float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kBlockN; ++c) {
-        const float x = (float)(int)s[c] * (cr * sc[c]);
-        s[c] = __float_as_uint(x);
-        if (c < vis) bmax = fmaxf(bmax, x);
+      for (int c = 0; c < 64; c += 2) {
+        const float x0 = (float)(int)s[c] * (cr * sc[c]);
+        const float x1 = (float)(int)s[c + 1] * (cr * sc[c + 1]);
+        s[c] = __float_as_uint(x0);
+        s[c + 1] = __float_as_uint(x1);
+        if (c < vis) mx0 = fmaxf(mx0, x0);
+        if (c + 1 < vis) mx1 = fmaxf(mx1, x1);
       }
-      const float m_new = fmaxf(m, bmax);
+      ctrl.red_max[j & 1][g][r] = fmaxf(mx0, mx1);
+      go = named_bar_and(kBarSoftmax, kSoftmaxThreads, ok);
+      if (!go) break;
+      const float m_new = fmaxf(m, fmaxf(ctrl.red_max[j & 1][0][r], ctrl.red_max[j & 1][1][r]));
       const float alpha = (m_new == -INFINITY || m == m_new) ? 1.f : (m == -INFINITY ? 0.f : fast_exp2(m - m_new));
-      uint32_t pc[32];
+      // P * 448 = 2^(x - (m_new - log2 448)): the scale to e4m3's range rides in the
+      // exponent's offset
+      const float moff = m_new - 8.8073549220576041f;
+      uint32_t pc[16];
       float lsum0 = 0.f, lsum1 = 0.f;
+      if (__all_sync(0xffffffffu, vis == 64)) {  // every key of the block visible (warp-uniform)
 #pragma unroll
-      for (int c = 0; c < kBlockN; c += 4) {
-        const float p0 = (c < vis) ? fast_exp2(__uint_as_float(s[c]) - m_new) * 448.f : 0.f;
-        const float p1 = (c + 1 < vis) ? fast_exp2(__uint_as_float(s[c + 1]) - m_new) * 448.f : 0.f;
-        const float p2 = (c + 2 < vis) ? fast_exp2(__uint_as_float(s[c + 2]) - m_new) * 448.f : 0.f;
-        const float p3 = (c + 3 < vis) ? fast_exp2(__uint_as_float(s[c + 3]) - m_new) * 448.f : 0.f;
-        const uint32_t lo = e4m3x2(p0, p1), hi = e4m3x2(p2, p3);
-        pc[c >> 2] = lo | (hi << 16);
-        lsum0 += e4m3x2_sum(lo);
-        lsum1 += e4m3x2_sum(hi);
+        for (int c = 0; c < 64; c += 4) {
+          const uint32_t lo = e4m3x2(fast_exp2(__uint_as_float(s[c]) - moff), fast_exp2(__uint_as_float(s[c + 1]) - moff));
+          const uint32_t hi =
+              e4m3x2(fast_exp2(__uint_as_float(s[c + 2]) - moff), fast_exp2(__uint_as_float(s[c + 3]) - moff));
+          pc[c >> 2] = lo | (hi << 16);
+          lsum0 = add_e4m3x2_to(lsum0, lo);
+          lsum1 = add_e4m3x2_to(lsum1, hi);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+          const float p0 = (c < vis) ? fast_exp2(__uint_as_float(s[c]) - moff) : 0.f;
+          const float p1 = (c + 1 < vis) ? fast_exp2(__uint_as_float(s[c + 1]) - moff) : 0.f;
+          const float p2 = (c + 2 < vis) ? fast_exp2(__uint_as_float(s[c + 2]) - moff) : 0.f;
+          const float p3 = (c + 3 < vis) ? fast_exp2(__uint_as_float(s[c + 3]) - moff) : 0.f;
+          const uint32_t lo = e4m3x2(p0, p1), hi = e4m3x2(p2, p3);
+          pc[c >> 2] = lo | (hi << 16);
+          lsum0 = add_e4m3x2_to(lsum0, lo);
+          lsum1 = add_e4m3x2_to(lsum1, hi);
+        }
       }
       l = l * alpha + (lsum0 + lsum1);
       m = m_new;
@@ -367,40 +395,43 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
       tc_fence_after();
       if (j > 0 && ok && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-        for (int c = 0; c < kDV; c += 32) {
+        for (int c = 0; c < 64; c += 32) {
           uint32_t o[32];
-          tmem_ld32(tmem + kTmemO + lane_off + c, o);
+          tmem_ld32(tmem + kTmemO + lane_off + 64 * g + c, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem + kTmemO + lane_off + c, o);
+          tmem_st32(tmem + kTmemO + lane_off + 64 * g + c, o);
         }
         tmem_wait_st();
       }
-      // P row r: 128 codes, 128-byte swizzle (16-byte granule g at g ^ (r & 7))
+      // P row r, keys 64g..64g+63: 16-byte granules 4g..4g+3 of the 128-byte row, swizzled
+      // (granule G at G ^ (r & 7))
       {
         const uint32_t prow = sP + r * kBlockN;
 #pragma unroll
-        for (int g = 0; g < 8; ++g)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + ((g ^ (r & 7)) << 4)),
-                       "r"(pc[4 * g]), "r"(pc[4 * g + 1]), "r"(pc[4 * g + 2]), "r"(pc[4 * g + 3])
+        for (int q = 0; q < 4; ++q)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + (((4 * g + q) ^ (r & 7)) << 4)),
+                       "r"(pc[4 * q]), "r"(pc[4 * q + 1]), "r"(pc[4 * q + 2]), "r"(pc[4 * q + 3])
                        : "memory");
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      go = named_bar_and(kBarSoftmax, kBlockM, ok);
-      if (go && r == 0) mbar_arrive(smem_u32(&ctrl.p_full));
+      go = named_bar_and(kBarSoftmax, kSoftmaxThreads, ok);
+      if (go && st == 0) mbar_arrive(smem_u32(&ctrl.p_full));
     }
     // epilogue after the last PV: out = O * s_v / l, lse = (m + log2(l / 448)) ln 2
     if (go) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), (nkb - 1) & 1) && ok;
     tc_fence_after();
-    go = named_bar_and(kBarSoftmax, kBlockM, ok && go);
+    ctrl.red_l[g][r] = l;
+    go = named_bar_and(kBarSoftmax, kSoftmaxThreads, ok && go);
     if (go) {
-      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      const float lrow = ctrl.red_l[0][r] + ctrl.red_l[1][r];
+      const float inv = (lrow > 0.f) ? 1.f / lrow : 0.f;
       const float* sv = p.sv + h * kDV;
       __nv_bfloat16* orow = p.out + ((int64_t)row * p.H + h) * kDV;
 #pragma unroll 1
-      for (int c = 0; c < kDV; c += 32) {
+      for (int c = 64 * g; c < 64 * g + 64; c += 32) {
         uint32_t o[32];
         tmem_ld32(tmem + kTmemO + lane_off + c, o);
         tmem_wait_ld();
@@ -417,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
             reinterpret_cast<uint4*>(orow + c)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (valid) p.lse[(int64_t)row * p.H + h] = (m + __log2f(l * (1.f / 448.f))) * 0.69314718055994531f;
+      if (valid && g == 0) p.lse[(int64_t)row * p.H + h] = (m + __log2f(lrow * (1.f / 448.f))) * 0.69314718055994531f;
     }
   }
 
