@@ -69,7 +69,7 @@ def prefill_work(S, H):
     return 2.0 * (192 + 128) * H * S * (S + 1) / 2
 
 
-def bench_prefill(mla, dev, steps, warmup):
+def bench_prefill(mla, dev, steps, warmup, S=None, H=None):
     """Quantised causal prefill (64K tokens, 16 heads, head dim 192) on seeded device
     inputs (N(0, 1) bf16 from a seeded torch generator; the inputs and the quantised
     workspace exceed L2).  Returns the per-workload entry: quantiser and attention
@@ -78,7 +78,8 @@ def bench_prefill(mla, dev, steps, warmup):
     import torch
     from deepseek_mla_decode_b200.workloads import PREFILL_S, PREFILL_H, PREFILL_SEED
 
-    S, H = PREFILL_S, PREFILL_H
+    S = S or PREFILL_S
+    H = H or PREFILL_H
     g = torch.Generator(device=dev).manual_seed(PREFILL_SEED)
     q = torch.randn((S, H, 192), generator=g, device=dev).to(torch.bfloat16)
     k = torch.randn((S, H, 192), generator=g, device=dev).to(torch.bfloat16)
@@ -460,6 +461,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--prefill-steps", type=int, default=5,
                     help="timed runs of the quantised 64K-token prefill (0 = skip)")
+    ap.add_argument("--prefill-shape", default="65536,16", help="S,H of the quantised prefill")
     ap.add_argument("--kv-format", default="bf16", choices=["bf16", "fp8"],
                     help="cache of the headline run: bf16 rows, or the packed FP8 rows (quantised once, untimed)")
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -597,7 +599,8 @@ def main():
             torch.cuda.empty_cache()
 
     if world == 1 and args.prefill_steps > 0:
-        per_workload["prefill_s65536_h16"] = bench_prefill(mla, dev, args.prefill_steps, 2)
+        pS, pH = (int(x) for x in args.prefill_shape.split(","))
+        per_workload[f"prefill_s{pS}_h{pH}"] = bench_prefill(mla, dev, args.prefill_steps, 2, pS, pH)
         torch.cuda.empty_cache()
 
     if rank != 0:
