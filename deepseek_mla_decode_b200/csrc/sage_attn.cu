@@ -13,15 +13,15 @@
 //   out_i  = O_acc * s_v / l,   lse_i = (m + log2(l / 448)) * ln 2
 // i.e. the output is normalised by the quantised weights that entered the product.
 //
-// One CTA = one head x 128 query rows.  Warp 0 issues the TMA loads (Q once; per key
-// block its K slab, V slab and the keys' scales), warp 1 the MMAs (QK of block j+1 is
-// issued before PV of block j, so the tensor core works while the softmax runs),
-// warps 4..11 the softmax and the epilogue (two threads per query row: warps 4..7 take
-// keys / output columns 0..63 of each block, warps 8..11 columns 64..127; a row's TMEM
-// lane is reachable from both, lane quadrant = warp % 4).
-// TMEM: S double buffer in columns [0, 256), O in [256, 384).  Every wait is bounded:
-// a timeout sets MLA_DEVICE_ERR_TIMEOUT, every role stops at its next wait, the CTA
-// drains its tensor-core work and returns.
+// One CTA = one head x two adjacent 128-row query tiles (rows 256 i .. 256 i + 255),
+// longest rows first.  Warp 0 issues the TMA loads (both tiles' Q once; per key block
+// its K slab, V slab and the keys' scales, shared by the two tiles), warp 1 the MMAs,
+// warps 4..7 the softmax of tile 0 and warps 8..11 that of tile 1 (one thread per
+// query row = TMEM lane).  The MMA order QK(0, j+1), PV(1, j), QK(1, j+1), PV(0, j+1)
+// ... lets one tile's softmax run while the tensor core works on the other tile.
+// TMEM: S of tile t in columns [128 t, 128 t + 128), O of tile t in [256 + 128 t, ...).
+// Every wait is bounded: a timeout sets MLA_DEVICE_ERR_TIMEOUT, every role stops at its
+// next wait, the CTA drains its tensor-core work and returns.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -39,22 +39,25 @@ using namespace ptx;
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kProducerWarp = 0, kMmaWarp = 1, kSoftmaxWarp0 = 4;
-constexpr int kSoftmaxThreads = 256;  // warps 4..11: two threads per query row, 64 keys each
-constexpr int kStages = 4;
+constexpr int kProducerWarp = 0, kMmaWarp = 1, kSoftmaxWarp0 = 4;  // tile t: warps 4 + 4t .. 7 + 4t
+constexpr int kTiles = 2;
+constexpr int kStages = 3;
 constexpr int kChunk = kBlockN * 64;          // one [128 rows][64 B] SW64 box (8 KB)
-constexpr int kQBytes = 3 * kChunk;           // Q: 128 rows x 192 B
+constexpr int kQBytes = 3 * kChunk;           // Q of a tile: 128 rows x 192 B
 constexpr int kKBytes = 3 * kChunk;           // K slab: 128 keys x 192 B
 constexpr int kVBytes = kDV * kBlockN;        // V slab: 128 channels x 128 keys (e4m3)
 constexpr int kStageBytes = kKBytes + kVBytes;  // 40 KB, a multiple of 1024
-constexpr int kPBytes = kBlockM * kBlockN;    // P: 128 rows x 128 keys (e4m3)
-constexpr int kSmemQ = 0, kSmemP = kSmemQ + kQBytes, kSmemStage = kSmemP + kPBytes;
+constexpr int kPBytes = kBlockM * kBlockN;    // P of a tile: 128 rows x 128 keys (e4m3)
+constexpr int kSmemQ = 0, kSmemP = kSmemQ + kTiles * kQBytes, kSmemStage = kSmemP + kTiles * kPBytes;
 constexpr int kSmemScale = kSmemStage + kStages * kStageBytes;
 constexpr int kSmemDyn = kSmemScale + kStages * kBlockN * 4;
 constexpr uint32_t kTmemS0 = 0, kTmemO = 256, kTmemCols = 512;
-constexpr int kBarSoftmax = 1;
 constexpr uint64_t kDrainWaitNs = 100000000ull;
 constexpr uint64_t kQuiesceNs = 500000ull;
+// setmaxnreg split: warps 0..3 (producer, MMA, two idle) give registers to the softmax
+// warpgroups; 128 x 56 + 256 x 224 = 384 x 168, the launch allocation.
+constexpr int kRegsIssue = 56, kRegsSoftmax = 224;
+static_assert(128 * kRegsIssue + 256 * kRegsSoftmax == kThreads * 168, "register split");
 
 // Instruction descriptor (D format, A/B formats, K-major A and B, N, M).
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t dfmt, uint32_t afmt, uint32_t bfmt, int M, int N) {
@@ -81,17 +84,15 @@ struct Params {
 
 struct __align__(8) Ctrl {
   uint64_t full[kStages];   // K, V and scales of a stage landed (count 1 + tx)
-  uint64_t empty[kStages];  // PV of the stage's block done (commit)
-  uint64_t q_full;
-  uint64_t s_full[2];       // S buffer written (commit)
-  uint64_t s_free[2];       // S buffer read by the 256 softmax threads
-  uint64_t p_full;          // P written and O rescaled (one arrive)
-  uint64_t p_free;          // PV done (commit)
+  uint64_t empty[kStages];  // both tiles' PV of the stage's block done (commit)
+  uint64_t q_full;          // both tiles' Q landed
+  uint64_t s_full[kTiles];  // S of a tile written (commit)
+  uint64_t s_free[kTiles];  // S of a tile read by its 128 softmax threads
+  uint64_t p_full[kTiles];  // P of a tile written and its O rescaled (one arrive)
+  uint64_t p_free[kTiles];  // PV of a tile done (commit)
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort;
-  float red_max[2][2][kBlockM];  // per block parity, column half, row: block maximum
-  float red_l[2][kBlockM];       // per column half, row: sum of coded weights
 };
 
 __device__ __forceinline__ void set_status(const Params& p, int bits) {
@@ -163,6 +164,14 @@ __device__ __forceinline__ bool named_bar_and(int id, int count, bool pred) {
       : "memory");
   return r != 0;
 }
+template <int kRegs>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <int kRegs>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -203,10 +212,15 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + kSmemQ, sP = sbase + kSmemP, sStage = sbase + kSmemStage, sScale = sbase + kSmemScale;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // longest rows first: work item w -> query block nqb - 1 - w / H, head w % H
-  const int qb = p.nqb - 1 - (int)(blockIdx.x / p.H);
+  // longest rows first: work item w -> tile pair npair - 1 - w / H, head w % H
+  const int npair = (p.nqb + 1) / 2;
+  const int pair = npair - 1 - (int)(blockIdx.x / p.H);
   const int h = (int)(blockIdx.x % p.H);
-  const int nkb = qb + 1;  // causal: key blocks 0..qb
+  const int qb0 = 2 * pair;
+  // causal: tile t (query block qb0 + t) sees key blocks 0..qb0 + t; a second tile past
+  // the last query block (odd block count) does nothing
+  const int nk0 = qb0 + 1, nk1 = (qb0 + 1 < p.nqb) ? qb0 + 2 : 0;
+  const int nkb = max(nk0, nk1);
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -214,12 +228,12 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
       mbar_init(smem_u32(&ctrl.empty[s]), 1);
     }
     mbar_init(smem_u32(&ctrl.q_full), 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(smem_u32(&ctrl.s_full[s]), 1);
-      mbar_init(smem_u32(&ctrl.s_free[s]), kSoftmaxThreads);
+    for (int t = 0; t < kTiles; ++t) {
+      mbar_init(smem_u32(&ctrl.s_full[t]), 1);
+      mbar_init(smem_u32(&ctrl.s_free[t]), kBlockM);
+      mbar_init(smem_u32(&ctrl.p_full[t]), 1);
+      mbar_init(smem_u32(&ctrl.p_free[t]), 1);
     }
-    mbar_init(smem_u32(&ctrl.p_full), 1);
-    mbar_init(smem_u32(&ctrl.p_free), 1);
     mbar_init(smem_u32(&ctrl.drain), 1);
     ctrl.abort = 0;
     fence_mbar_init();
@@ -244,10 +258,14 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
     // =====================================================================
     // TMA producer (lane 0 issues; the warp waits together)
     // =====================================================================
+    regs_dec<kRegsIssue>();
     bool ok = true;
     if (lane == 0) {
-      expect_tx(smem_u32(&ctrl.q_full), kQBytes);
-      for (int c = 0; c < 3; ++c) tma_3d(sQ + c * kChunk, &p.tm_q, smem_u32(&ctrl.q_full), 64 * c, qb * kBlockM, h);
+      const int ntiles = nk1 > 0 ? 2 : 1;
+      expect_tx(smem_u32(&ctrl.q_full), ntiles * kQBytes);
+      for (int t = 0; t < ntiles; ++t)
+        for (int c = 0; c < 3; ++c)
+          tma_3d(sQ + t * kQBytes + c * kChunk, &p.tm_q, smem_u32(&ctrl.q_full), 64 * c, (qb0 + t) * kBlockM, h);
     }
     for (int j = 0; j < nkb && ok; ++j) {
       const int st = j % kStages, use = j / kStages;
@@ -265,8 +283,10 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
     }
   } else if (warp == kMmaWarp) {
     // =====================================================================
-    // MMA issuer: QK(0), then QK(j + 1) before PV(j)
+    // MMA issuer: QK(0, 0), QK(1, 0), then per key block j: PV(0, j), QK(0, j + 1),
+    // PV(1, j), QK(1, j + 1), and the block's stage is released
     // =====================================================================
+    regs_dec<kRegsIssue>();
     bool ok = wait_bar(&ctrl, p, smem_u32(&ctrl.q_full), 0);
     const bool elected = elect_one();
     // K-major operands: Q / K slabs are three [128 rows][64 B] boxes with the 64-byte
@@ -277,77 +297,89 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
     const uint64_t dk0 = make_smem_desc(sStage, 16, 512, kSwizzle64B);
     const uint64_t dv0 = make_smem_desc(sStage + kKBytes, 16, 1024, kSwizzle128B);
     const uint64_t dp0 = make_smem_desc(sP, 16, 1024, kSwizzle128B);
-    constexpr uint64_t kChunkD = kChunk >> 4, kStageD = kStageBytes >> 4;
-    auto qk = [&](int j) {
+    constexpr uint64_t kChunkD = kChunk >> 4, kStageD = kStageBytes >> 4, kQD = kQBytes >> 4, kPD = kPBytes >> 4;
+    auto qk = [&](int t, int j) {
       const int st = j % kStages;
       ok = ok && wait_bar(&ctrl, p, smem_u32(&ctrl.full[st]), (j / kStages) & 1);
-      if (ok && j >= 2) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.s_free[j & 1]), ((j >> 1) - 1) & 1);
+      if (ok && j >= 1) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.s_free[t]), (j - 1) & 1);
       if (!ok) return;
       tc_fence_after();
       if (elected) {
 #pragma unroll
         for (int ks = 0; ks < 6; ++ks) {
           const uint64_t off = (ks >> 1) * kChunkD + (ks & 1) * 2;
-          mma_i8(tmem + kTmemS0 + 128 * (j & 1), dq0 + off, dk0 + st * kStageD + off, kIdescQK, ks > 0);
+          mma_i8(tmem + kTmemS0 + 128 * t, dq0 + t * kQD + off, dk0 + st * kStageD + off, kIdescQK, ks > 0);
         }
-        commit(smem_u32(&ctrl.s_full[j & 1]));
+        commit(smem_u32(&ctrl.s_full[t]));
       }
       __syncwarp();
     };
-    auto pv = [&](int j) {
+    auto pv = [&](int t, int j) {
       const int st = j % kStages;
-      ok = ok && wait_bar(&ctrl, p, smem_u32(&ctrl.p_full), j & 1);
+      ok = ok && wait_bar(&ctrl, p, smem_u32(&ctrl.p_full[t]), j & 1);
       if (!ok) return;
       tc_fence_after();
       if (elected) {
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_f8(tmem + kTmemO, dp0 + ks * 2, dv0 + st * kStageD + ks * 2, kIdescPV, (j > 0 || ks > 0));
-        commit(smem_u32(&ctrl.empty[st]));
-        commit(smem_u32(&ctrl.p_free));
+          mma_f8(tmem + kTmemO + 128 * t, dp0 + t * kPD + ks * 2, dv0 + st * kStageD + ks * 2, kIdescPV,
+                 (j > 0 || ks > 0));
+        commit(smem_u32(&ctrl.p_free[t]));
       }
       __syncwarp();
     };
-    qk(0);
+    qk(0, 0);
+    if (nk1 > 0) qk(1, 0);
     for (int j = 0; j < nkb && ok; ++j) {
-      if (j + 1 < nkb) qk(j + 1);
-      pv(j);
+#pragma unroll
+      for (int t = 0; t < kTiles; ++t) {
+        const int nkt = t == 0 ? nk0 : nk1;
+        if (j < nkt) {
+          pv(t, j);
+          if (j + 1 < nkt) qk(t, j + 1);
+        }
+      }
+      if (ok && elected) commit(smem_u32(&ctrl.empty[j % kStages]));  // after both tiles' PV of block j
+      __syncwarp();
     }
   } else if (warp >= kSoftmaxWarp0) {
     // =====================================================================
-    // softmax + epilogue: thread (g, r) = query row r (TMEM lane r), columns 64g..64g+63
+    // softmax + epilogue: tile t, thread = query row r of the tile (TMEM lane r)
     // =====================================================================
-    const int st = tid - kSoftmaxWarp0 * 32;  // 0..255
-    const int g = st >> 7, r = st & 127;
+    regs_inc<kRegsSoftmax>();
+    const int t = (warp - kSoftmaxWarp0) >> 2;
+    const int r = tid - (kSoftmaxWarp0 + 4 * t) * 32;  // 0..127
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const int row = qb * kBlockM + r;
+    const int row = (qb0 + t) * kBlockM + r;
+    const int nkt = t == 0 ? nk0 : nk1;
     const bool valid = row < p.S;
     const float cr = valid ? p.sq[(int64_t)h * p.S_pad + row] * p.scale_log2 : 0.f;
+    const uint32_t sPt = sP + t * kPBytes;
+    const uint32_t tS = tmem + kTmemS0 + 128 * t + lane_off, tO = tmem + kTmemO + 128 * t + lane_off;
     float m = -INFINITY, l = 0.f;
-    bool ok = true, go = true;
+    bool ok = true, go = nkt > 0;
     const float* sc_all = reinterpret_cast<const float*>(smem + kSmemScale);
-    for (int j = 0; j < nkb && go; ++j) {
+    for (int j = 0; j < nkt && go; ++j) {
       const int stg = j % kStages;
-      ok = wait_bar(&ctrl, p, smem_u32(&ctrl.s_full[j & 1]), (j >> 1) & 1) && ok;
+      ok = wait_bar(&ctrl, p, smem_u32(&ctrl.s_full[t]), j & 1) && ok;
       // the stage's scales landed with its TMA (already complete; this wait makes them
       // visible to these threads)
       ok = wait_bar(&ctrl, p, smem_u32(&ctrl.full[stg]), (j / kStages) & 1) && ok;
       tc_fence_after();
-      uint32_t s[64];
+      uint32_t s[128];
       if (ok) {
-        const uint32_t ta = tmem + kTmemS0 + 128 * (j & 1) + lane_off + 64 * g;
-        tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
         tmem_wait_ld();
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&ctrl.s_free[j & 1]));  // the S buffer may be overwritten
-      // dequantised log2-scaled scores of the visible keys (key j*128 + 64g + c <= row)
-      const float* sc = sc_all + stg * kBlockN + 64 * g;
-      const int vis = valid ? max(0, min(64, row - j * kBlockN - 64 * g + 1)) : 0;
+      mbar_arrive(smem_u32(&ctrl.s_free[t]));  // S of this tile may be overwritten
+      // dequantised log2-scaled scores of the visible keys (key j*128 + c <= row)
+      const float* sc = sc_all + stg * kBlockN;
+      const int vis = valid ? max(0, min(kBlockN, row - j * kBlockN + 1)) : 0;
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
+      for (int c = 0; c < kBlockN; c += 2) {
         const float x0 = (float)(int)s[c] * (cr * sc[c]);
         const float x1 = (float)(int)s[c + 1] * (cr * sc[c + 1]);
         s[c] = __float_as_uint(x0);
@@ -355,19 +387,16 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
         if (c < vis) mx0 = fmaxf(mx0, x0);
         if (c + 1 < vis) mx1 = fmaxf(mx1, x1);
       }
-      ctrl.red_max[j & 1][g][r] = fmaxf(mx0, mx1);
-      go = named_bar_and(kBarSoftmax, kSoftmaxThreads, ok);
-      if (!go) break;
-      const float m_new = fmaxf(m, fmaxf(ctrl.red_max[j & 1][0][r], ctrl.red_max[j & 1][1][r]));
+      const float m_new = fmaxf(m, fmaxf(mx0, mx1));
       const float alpha = (m_new == -INFINITY || m == m_new) ? 1.f : (m == -INFINITY ? 0.f : fast_exp2(m - m_new));
       // P * 448 = 2^(x - (m_new - log2 448)): the scale to e4m3's range rides in the
       // exponent's offset
       const float moff = m_new - 8.8073549220576041f;
-      uint32_t pc[16];
+      uint32_t pc[32];
       float lsum0 = 0.f, lsum1 = 0.f;
-      if (__all_sync(0xffffffffu, vis == 64)) {  // every key of the block visible (warp-uniform)
+      if (__all_sync(0xffffffffu, vis == kBlockN)) {  // every key of the block visible (warp-uniform)
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) {
+        for (int c = 0; c < kBlockN; c += 4) {
           const uint32_t lo = e4m3x2(fast_exp2(__uint_as_float(s[c]) - moff), fast_exp2(__uint_as_float(s[c + 1]) - moff));
           const uint32_t hi =
               e4m3x2(fast_exp2(__uint_as_float(s[c + 2]) - moff), fast_exp2(__uint_as_float(s[c + 3]) - moff));
@@ -377,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) {
+        for (int c = 0; c < kBlockN; c += 4) {
           const float p0 = (c < vis) ? fast_exp2(__uint_as_float(s[c]) - moff) : 0.f;
           const float p1 = (c + 1 < vis) ? fast_exp2(__uint_as_float(s[c + 1]) - moff) : 0.f;
           const float p2 = (c + 2 < vis) ? fast_exp2(__uint_as_float(s[c + 2]) - moff) : 0.f;
@@ -390,50 +419,48 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
       }
       l = l * alpha + (lsum0 + lsum1);
       m = m_new;
-      // PV of the previous block must be done before P is overwritten or O rescaled
-      if (j > 0) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), (j - 1) & 1) && ok;
+      // PV of this tile's previous block must be done before P is overwritten or O
+      // rescaled
+      if (j > 0) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free[t]), (j - 1) & 1) && ok;
       tc_fence_after();
       if (j > 0 && ok && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-        for (int c = 0; c < 64; c += 32) {
+        for (int c = 0; c < kDV; c += 32) {
           uint32_t o[32];
-          tmem_ld32(tmem + kTmemO + lane_off + 64 * g + c, o);
+          tmem_ld32(tO + c, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem + kTmemO + lane_off + 64 * g + c, o);
+          tmem_st32(tO + c, o);
         }
         tmem_wait_st();
       }
-      // P row r, keys 64g..64g+63: 16-byte granules 4g..4g+3 of the 128-byte row, swizzled
-      // (granule G at G ^ (r & 7))
+      // P row r: 128 codes, 128-byte swizzle (16-byte granule g at g ^ (r & 7))
       {
-        const uint32_t prow = sP + r * kBlockN;
+        const uint32_t prow = sPt + r * kBlockN;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + (((4 * g + q) ^ (r & 7)) << 4)),
-                       "r"(pc[4 * q]), "r"(pc[4 * q + 1]), "r"(pc[4 * q + 2]), "r"(pc[4 * q + 3])
+        for (int g = 0; g < 8; ++g)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + ((g ^ (r & 7)) << 4)),
+                       "r"(pc[4 * g]), "r"(pc[4 * g + 1]), "r"(pc[4 * g + 2]), "r"(pc[4 * g + 3])
                        : "memory");
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      go = named_bar_and(kBarSoftmax, kSoftmaxThreads, ok);
-      if (go && st == 0) mbar_arrive(smem_u32(&ctrl.p_full));
+      go = named_bar_and(1 + t, kBlockM, ok);
+      if (go && r == 0) mbar_arrive(smem_u32(&ctrl.p_full[t]));
     }
-    // epilogue after the last PV: out = O * s_v / l, lse = (m + log2(l / 448)) ln 2
-    if (go) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), (nkb - 1) & 1) && ok;
+    // epilogue after the tile's last PV: out = O * s_v / l, lse = (m + log2(l / 448)) ln 2
+    if (go) ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free[t]), (nkt - 1) & 1) && ok;
     tc_fence_after();
-    ctrl.red_l[g][r] = l;
-    go = named_bar_and(kBarSoftmax, kSoftmaxThreads, ok && go);
+    if (nkt > 0) go = named_bar_and(1 + t, kBlockM, ok && go);
     if (go) {
-      const float lrow = ctrl.red_l[0][r] + ctrl.red_l[1][r];
-      const float inv = (lrow > 0.f) ? 1.f / lrow : 0.f;
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
       const float* sv = p.sv + h * kDV;
       __nv_bfloat16* orow = p.out + ((int64_t)row * p.H + h) * kDV;
 #pragma unroll 1
-      for (int c = 64 * g; c < 64 * g + 64; c += 32) {
+      for (int c = 0; c < kDV; c += 32) {
         uint32_t o[32];
-        tmem_ld32(tmem + kTmemO + lane_off + c, o);
+        tmem_ld32(tO + c, o);
         tmem_wait_ld();
         if (valid) {
           uint32_t w[16];
@@ -448,8 +475,10 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
             reinterpret_cast<uint4*>(orow + c)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (valid && g == 0) p.lse[(int64_t)row * p.H + h] = (m + __log2f(lrow * (1.f / 448.f))) * 0.69314718055994531f;
+      if (valid) p.lse[(int64_t)row * p.H + h] = (m + __log2f(l * (1.f / 448.f))) * 0.69314718055994531f;
     }
+  } else {
+    regs_dec<kRegsIssue>();  // the idle warps of the first warpgroup
   }
 
   // ---- teardown ------------------------------------------------------------
@@ -506,7 +535,7 @@ cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, c
   prm.H = H;
   prm.nqb = prm.S_pad / kBlockM;
   prm.scale_log2 = softmax_scale * 1.4426950408889634f;
-  const unsigned grid = (unsigned)prm.nqb * (unsigned)H;
+  const unsigned grid = (unsigned)((prm.nqb + 1) / 2) * (unsigned)H;
   sage_attn_kernel<<<grid, kThreads, kSmemDyn + 1024, stream>>>(prm);
   return cudaGetLastError();
 }
