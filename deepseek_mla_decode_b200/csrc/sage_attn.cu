@@ -374,20 +374,22 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&ctrl.s_free[t]));  // S of this tile may be overwritten
-      // dequantised log2-scaled scores of the visible keys (key j*128 + c <= row)
+      // key-scaled scores x' = S_int * s_k of the visible keys (key j*128 + c <= row); the
+      // row factor cr = s_q * scale * log2(e) > 0 (or 0 for a zero or invalid row) keeps
+      // their order, so it is applied once to the maximum and inside the exponent's FMA
       const float* sc = sc_all + stg * kBlockN;
       const int vis = valid ? max(0, min(kBlockN, row - j * kBlockN + 1)) : 0;
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
       for (int c = 0; c < kBlockN; c += 2) {
-        const float x0 = (float)(int)s[c] * (cr * sc[c]);
-        const float x1 = (float)(int)s[c + 1] * (cr * sc[c + 1]);
+        const float x0 = (float)(int)s[c] * sc[c];
+        const float x1 = (float)(int)s[c + 1] * sc[c + 1];
         s[c] = __float_as_uint(x0);
         s[c + 1] = __float_as_uint(x1);
         if (c < vis) mx0 = fmaxf(mx0, x0);
         if (c + 1 < vis) mx1 = fmaxf(mx1, x1);
       }
-      const float m_new = fmaxf(m, fmaxf(mx0, mx1));
+      const float m_new = fmaxf(m, vis > 0 ? cr * fmaxf(mx0, mx1) : -INFINITY);
       const float alpha = (m_new == -INFINITY || m == m_new) ? 1.f : (m == -INFINITY ? 0.f : fast_exp2(m - m_new));
       // P * 448 = 2^(x - (m_new - log2 448)): the scale to e4m3's range rides in the
       // exponent's offset
@@ -397,9 +399,9 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
       if (__all_sync(0xffffffffu, vis == kBlockN)) {  // every key of the block visible (warp-uniform)
 #pragma unroll
         for (int c = 0; c < kBlockN; c += 4) {
-          const uint32_t lo = e4m3x2(fast_exp2(__uint_as_float(s[c]) - moff), fast_exp2(__uint_as_float(s[c + 1]) - moff));
+          const uint32_t lo = e4m3x2(fast_exp2(fmaf(__uint_as_float(s[c]), cr, -moff)), fast_exp2(fmaf(__uint_as_float(s[c + 1]), cr, -moff)));
           const uint32_t hi =
-              e4m3x2(fast_exp2(__uint_as_float(s[c + 2]) - moff), fast_exp2(__uint_as_float(s[c + 3]) - moff));
+              e4m3x2(fast_exp2(fmaf(__uint_as_float(s[c + 2]), cr, -moff)), fast_exp2(fmaf(__uint_as_float(s[c + 3]), cr, -moff)));
           pc[c >> 2] = lo | (hi << 16);
           lsum0 = add_e4m3x2_to(lsum0, lo);
           lsum1 = add_e4m3x2_to(lsum1, hi);
@@ -407,10 +409,10 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
       } else {
 #pragma unroll
         for (int c = 0; c < kBlockN; c += 4) {
-          const float p0 = (c < vis) ? fast_exp2(__uint_as_float(s[c]) - moff) : 0.f;
-          const float p1 = (c + 1 < vis) ? fast_exp2(__uint_as_float(s[c + 1]) - moff) : 0.f;
-          const float p2 = (c + 2 < vis) ? fast_exp2(__uint_as_float(s[c + 2]) - moff) : 0.f;
-          const float p3 = (c + 3 < vis) ? fast_exp2(__uint_as_float(s[c + 3]) - moff) : 0.f;
+          const float p0 = (c < vis) ? fast_exp2(fmaf(__uint_as_float(s[c]), cr, -moff)) : 0.f;
+          const float p1 = (c + 1 < vis) ? fast_exp2(fmaf(__uint_as_float(s[c + 1]), cr, -moff)) : 0.f;
+          const float p2 = (c + 2 < vis) ? fast_exp2(fmaf(__uint_as_float(s[c + 2]), cr, -moff)) : 0.f;
+          const float p3 = (c + 3 < vis) ? fast_exp2(fmaf(__uint_as_float(s[c + 3]), cr, -moff)) : 0.f;
           const uint32_t lo = e4m3x2(p0, p1), hi = e4m3x2(p2, p3);
           pc[c >> 2] = lo | (hi << 16);
           lsum0 = add_e4m3x2_to(lsum0, lo);
