@@ -131,3 +131,27 @@ def test_fp8_full_size_whole_batch(name):
     inp = make_workload(name)
     stats = check_fp8(inp, seqs=list(range(inp.B)))
     print(f"fp8 {name}: {stats}")
+
+
+def test_fp8_wait_timeout_sets_status_and_returns():
+    """The failure path of the FP8 instantiation: the MMA warp waits on a barrier nothing
+    completes (a test hook), bounded by 1 ms; converters and producers then stop at their
+    next bounded wait, the pair drains and returns, and the next call is exact."""
+    from mla_testlib import to_device
+
+    inp = make_inputs(3, 1, 128, [3000, 700, 5000], seed=371)
+    dev = to_device(inp)
+    kv8 = mla.quantize_kv_fp8(dev["kv_cache"])
+    meta = mla.get_metadata(dev["cache_seqlens"], 1, 128)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    try:
+        mla.set_wait_timeout_ns(1_000_000)
+        mla.set_stall_injection(True)
+        mla.decode_fp8(dev["q_nope"], dev["q_pe"], kv8, dev["block_table"], dev["cache_seqlens"],
+                       inp.softmax_scale, False, meta, status=status)
+        torch.cuda.synchronize()
+    finally:
+        mla.set_stall_injection(False)
+        mla.set_wait_timeout_ns(0)
+    assert int(status.item()) & mla.MLA_DEVICE_ERR_TIMEOUT
+    check_fp8(inp)
