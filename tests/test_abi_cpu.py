@@ -64,3 +64,29 @@ def test_null_pointers_rejected_before_any_device_call():
     rc = L.mla_get_metadata(None, 1, 1, 16, None, 0, None)
     assert rc == 1
     assert L.mla_metadata_size(1, 1, 16, None) == 1
+
+
+def test_fp8_and_prefill_entry_points_validate_before_any_device_call():
+    L = mla.load_library()
+    rc = L.mla_decode_fp8(None, None, None, 1, None, 1, None, None, 1, 1, 16, 0.1, 0, None, 0, None, 0, None, None,
+                          None, None)
+    assert rc == 1
+    rc = L.mla_decode_fp8_attention(None, None, None, 1, None, 1, None, None, 1, 1, 16, 0.1, 0, None, 0, None, 0,
+                                    None, None, None, None)
+    assert rc == 1
+    assert L.mla_quantize_kv_fp8(None, None, 1, None) == 1
+    n = ctypes.c_size_t()
+    assert L.mla_sage_workspace_size(0, 1, ctypes.byref(n)) == 1
+    assert L.mla_sage_workspace_size(1, 0, ctypes.byref(n)) == 1
+    assert L.mla_sage_workspace_size(1, 1, None) == 1
+    assert L.mla_sage_quantize(None, None, None, 10, 2, None, 0, None) == 1
+    assert L.mla_sage_attention(10, 2, 0.1, None, 0, None, None, None, None) == 1
+    assert L.mla_sage_prefill(None, None, None, 10, 2, 0.1, None, 0, None, None, None, None) == 1
+
+
+def test_prefill_workspace_size_host_only():
+    # codes (2 x 192 + 128 bytes per token and head, tokens padded to 128) + token scales
+    # (8 bytes per token and head) + channel scale and scratch (8 bytes per channel and head)
+    S, H = 300, 3
+    sp = 384
+    assert mla.sage_workspace_size(S, H) == H * sp * (2 * 192 + 128) + 2 * H * sp * 4 + 2 * H * 128 * 4
