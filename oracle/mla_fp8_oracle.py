@@ -12,8 +12,7 @@ Sources (page titles and sections):
 * A quantised KV cache scaled per token by its max-abs value: "DeepSeek speed test"
   article, section 3.1 (per-token INT8 KV).
 
-The pages give no FP8 cache format.  The readings taken here (each is listed in
-DESIGN.md):
+The pages give no FP8 cache format.  The readings taken here (this library's own):
 
 1. One fp32 scale per token (per cache row) for the whole 576-wide row:
    ``scale = amax / 448`` with ``amax = max |row|`` over c_kv and k_pe, and 448 the

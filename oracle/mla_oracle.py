@@ -28,7 +28,7 @@ What is computed (sources, by page title and section):
   outputs are merged by their log-sum-exp -- "DeepSeek speed test" article 2.1
   ("split-K parallelism"); the merge identity is exact algebra.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent (this library's own; each is stated here):
 V is the first 512 columns of the same cache row; lse uses the natural log and
 includes the scale; rows with no visible key give out = 0 and lse = -inf; block-table
 entries past ceil(n/64) and rows past n in the last block are never read.

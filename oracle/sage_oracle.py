@@ -12,7 +12,7 @@ dequantised, then an online softmax runs; its weights P are quantised to FP8 and
 multiplied with the FP8 V, and the product is dequantised by V's scale.  DeepSeek's
 case is a head dimension of 192 (128 without RoPE + 64 RoPE) for Q and K; V has 128.
 
-Readings where the page is silent (each is listed in the design doc):
+Readings where the page is silent (this library's own; each is stated here):
 
 1. Q and K are quantised per (token, head): ``s = max|x| / 127`` over the 192 values,
    ``code = round-half-even(x / s)``, scale and quotient in IEEE fp32; a zero row has
