@@ -85,9 +85,11 @@ def quantize_v_channels(v: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
 
 
 def sage_prefill_ref(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray,
-                     softmax_scale: float = SCALE_192) -> Tuple[np.ndarray, np.ndarray]:
+                     softmax_scale: float = SCALE_192, rows=None) -> Tuple[np.ndarray, np.ndarray]:
     """Quantised causal prefill attention.  q, k: bf16 bits [S, H, 192]; v: bf16 bits
-    [S, H, 128].  Returns (out float64 [S, H, 128], lse float64 [S, H])."""
+    [S, H, 128].  Returns (out float64 [R, H, 128], lse float64 [R, H]) for the query
+    rows ``rows`` (all S rows when None); each row follows the same steps whether or not
+    the others are computed (the quantisation scales still come from every token)."""
     q = F.O.bf16_to_f64(q_bits).astype(np.float32)
     k = F.O.bf16_to_f64(k_bits).astype(np.float32)
     v = F.O.bf16_to_f64(v_bits).astype(np.float32)
@@ -97,21 +99,23 @@ def sage_prefill_ref(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray,
     kc, sk = quantize_int8_rows(k)
     vc, sv = quantize_v_channels(v)
     v_hat = F.e4m3_decode(vc) * sv.astype(np.float64)[None]  # [S, H, 128]
-    out = np.zeros((S, H, D_V))
-    lse = np.zeros((S, H))
-    rows = np.arange(S)
+    rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    R = rows.size
+    out = np.zeros((R, H, D_V))
+    lse = np.zeros((R, H))
+    last = int(rows.max()) + 1 if R else 0  # keys past the last row are never visible
     for h in range(H):
         # exact integer scores (int64 accumulation of int8 products)
-        s_int = qc[:, h, :].astype(np.int64) @ kc[:, h, :].astype(np.int64).T  # [S, S]
-        logits = s_int.astype(np.float64) * sq[:, h].astype(np.float64)[:, None] \
-            * sk[:, h].astype(np.float64)[None, :] * softmax_scale
-        m = np.full(S, -np.inf)
-        l = np.zeros(S)
-        acc = np.zeros((S, D_V))
-        for b0 in range(0, S, KEY_BLOCK):
-            cols = np.arange(b0, min(b0 + KEY_BLOCK, S))
+        s_int = qc[rows, h, :].astype(np.int64) @ kc[:last, h, :].astype(np.int64).T  # [R, last]
+        logits = s_int.astype(np.float64) * sq[rows, h].astype(np.float64)[:, None] \
+            * sk[:last, h].astype(np.float64)[None, :] * softmax_scale
+        m = np.full(R, -np.inf)
+        l = np.zeros(R)
+        acc = np.zeros((R, D_V))
+        for b0 in range(0, last, KEY_BLOCK):
+            cols = np.arange(b0, min(b0 + KEY_BLOCK, last))
             live = rows >= b0  # rows that see at least one key of this block
-            blk = logits[:, cols]
+            blk = logits[:, b0:b0 + cols.size]
             vis = cols[None, :] <= rows[:, None]
             blk_max = np.where(vis, blk, -np.inf).max(axis=1)
             m_new = np.where(live, np.maximum(m, blk_max), m)

@@ -133,3 +133,26 @@ def test_sage_host_argument_errors():
     assert L.mla_sage_attention(10, 2, 0.1, ws.data_ptr(), n.value - 1, out.data_ptr(), lse.data_ptr(), None, None) != 0
     assert L.mla_sage_attention(10, 2, 0.1, ws.data_ptr(), n.value, None, lse.data_ptr(), None, None) != 0
     assert L.mla_sage_attention(10, 2, -1.0, ws.data_ptr(), n.value, out.data_ptr(), lse.data_ptr(), None, None) != 0
+
+
+def test_prefill_full_size_sampled_rows():
+    # the bench's configuration (64K tokens, 16 heads): rows sampled across the whole
+    # sequence (first and last rows, block and tile-pair edges, random interior rows)
+    # against the oracle, which computes each sampled row on its own
+    from deepseek_mla_decode_b200.workloads import make_prefill, PREFILL_S, PREFILL_H
+
+    S, H = PREFILL_S, PREFILL_H
+    q, k, v = make_prefill(S, H, seed=41)
+    out, lse = mla.sage_prefill(dev(q), dev(k), dev(v), SA.SCALE_192)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(42)
+    rows = sorted(set([0, 1, 127, 128, 255, 256, 257, 4095, 32767, 32768, S - 129, S - 128, S - 2, S - 1]
+                      + rng.integers(0, S, 34).tolist()))
+    ref, ref_lse = SA.sage_prefill_ref(q, k, v, rows=rows)
+    got = out[rows].float().cpu().double().numpy()
+    got_lse = lse[rows].cpu().double().numpy()
+    err = np.abs(got - ref)
+    stats = dict(out_max=float(err.max()), out_mean=float(err.mean()),
+                 lse_max=float(np.abs(got_lse - ref_lse).max()))
+    assert stats["out_max"] <= 2e-2 and stats["out_mean"] <= 2e-3 and stats["lse_max"] <= 1e-3, stats
+    print(stats)

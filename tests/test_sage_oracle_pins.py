@@ -201,3 +201,14 @@ def test_running_max_rescale_closed_form():
     assert np.allclose(out[128:], num / den, rtol=1e-12, atol=1e-12)
     assert np.allclose(lse[128:, 0], 2 * L + np.log(128 * r + (i - 127)), rtol=1e-12, atol=1e-12)
     assert np.allclose(out[:128], np.cumsum(v[:128], axis=0) / np.arange(1, 129)[:, None, None], rtol=1e-12)
+
+
+def test_row_subset_follows_the_same_steps():
+    # a subset of query rows gives exactly those rows of the full computation
+    rng = np.random.default_rng(9)
+    S, H = 333, 2
+    q, k, v = rand_bf16(rng, (S, H, 192)), rand_bf16(rng, (S, H, 192)), rand_bf16(rng, (S, H, 128))
+    out, lse = SA.sage_prefill_ref(q, k, v)
+    rows = [0, 1, 127, 128, 200, 255, 256, 332]
+    o2, l2 = SA.sage_prefill_ref(q, k, v, rows=rows)
+    assert np.array_equal(o2, out[rows]) and np.array_equal(l2, lse[rows])
