@@ -74,7 +74,7 @@ constexpr int kStgPerQk = 8 + 2;                   // raw stages per tile for QK
 // FP8 kernel register split (setmaxnreg, per warpgroup): warps 0-3 (producers, MMA),
 // 4-11 (softmax), 12-15 (converters); 128 x (issue + conv) + 256 x softmax must equal
 // the 512 x 128 registers the block is launched with.
-constexpr int kRegsIssue = 88, kRegsConv = 72, kRegsSoftmax = 176;
+constexpr int kRegsIssue = 88, kRegsConv = 88, kRegsSoftmax = 168;
 static_assert(128 * (kRegsIssue + kRegsConv) + 256 * kRegsSoftmax == 512 * 128, "register split");
 
 template <bool kFp8>
@@ -1244,7 +1244,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
         // Eight consecutive threads cover two rows x four granules: 128 contiguous raw
         // bytes and eight distinct swizzled granules, so neither side has bank conflicts.
         auto conv_slab = [&](const uint8_t* src, uint8_t* dst, int own) {
-#pragma unroll 2
+#pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int u = ct + kNumConvThreads * i, b = u >> 8;
             if (b >= own) continue;
@@ -1264,7 +1264,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
         // swizzled boxes (columns 0..63, 64..127).  Unit u: row m = u & 63, 16-column
         // granule k = u >> 6; eight consecutive threads take eight rows of one granule.
         auto conv_vslab = [&](const uint8_t* src, uint8_t* dst) {
-#pragma unroll 2
+#pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int u = ct + kNumConvThreads * i;
             const int m = u & 63, k = u >> 6;
