@@ -92,7 +92,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only whe
 constexpr uint32_t kIdescQK = make_idesc_bf16(128, 256, false, false);
 constexpr uint32_t kIdescPV = make_idesc_bf16(128, 256, false, true);
 constexpr int kBarSoftmax = 1;  // named barrier id for the 256 softmax threads
-constexpr int kBarConv = 2;     // named barrier id for the 128 converter threads
+constexpr int kBarConv = 2;     // named barrier ids 2, 3 for the two converter groups
 constexpr uint64_t kDrainWaitNs = 100000000ull;  // bound on the post-abort wait for tensor-core work
 constexpr uint64_t kQuiesceNs = 500000ull;       // post-abort wait for TMA loads in flight
 
@@ -1210,7 +1210,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
       if constexpr (kFp8) {
         regs_dec<kRegsConv>();
         constexpr int kStg = C::kStg;
-        const int ct = tid - kConvWarp0 * 32;  // 0..127
+        // two groups of two warps take alternate ring slots, so one group's hand-off
+        // overlaps the other group's conversion
+        const int grp = (tid - kConvWarp0 * 32) >> 6;  // 0, 1
+        const int ct = (tid - kConvWarp0 * 32) & 63;   // 0..63 within the group
+        constexpr int kGrpThreads = 64;
         PieceWalker walk(p, part, tile_row0);
         uint32_t js = 0, ir = 0;  // raw stages and ring slots consumed so far
         bool ok = true, go = true;
@@ -1226,7 +1230,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
         // together.
         auto publish = [&](uint32_t j0, int nraw) -> bool {
           fence_proxy_async_smem();
-          go = named_bar_and(kBarConv, kNumConvThreads, ok);
+          go = named_bar_and(kBarConv + grp, kGrpThreads, ok);
           if (!go) return false;
           if (ct == 0) {
             for (int k = 0; k < nraw; ++k) mbar_arrive(smem_u32(&ctrl.stg_empty[(j0 + k) % kStg]));
@@ -1245,8 +1249,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
         // bytes and eight distinct swizzled granules, so neither side has bank conflicts.
         auto conv_slab = [&](const uint8_t* src, uint8_t* dst, int own) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int u = ct + kNumConvThreads * i, b = u >> 8;
+          for (int i = 0; i < 8; ++i) {
+            const int u = ct + kGrpThreads * i, b = u >> 8;
             if (b >= own) continue;
             const int m = (u >> 2) & 63, k = u & 3;
             const uint4 v = *reinterpret_cast<const uint4*>(src + b * kSlabBlockBytes + m * 64 + 16 * k);
@@ -1265,8 +1269,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
         // granule k = u >> 6; eight consecutive threads take eight rows of one granule.
         auto conv_vslab = [&](const uint8_t* src, uint8_t* dst) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int u = ct + kNumConvThreads * i;
+          for (int i = 0; i < 8; ++i) {
+            const int u = ct + kGrpThreads * i;
             const int m = u & 63, k = u >> 6;
             const uint4 v = *reinterpret_cast<const uint4*>(src + m * 128 + ((k ^ (m & 7)) << 4));
             uint8_t* row = dst + (k >> 2) * kChunkBytes + m * 128;
@@ -1284,6 +1288,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
         auto conv_qk = [&](const Piece& pc, int t) {
           const int own = min(max(blocks_in_tile(pc, t) - 2 * (int)rank, 0), 2);
           for (int c = 0; c < 8; ++c) {
+            if ((int)(ir & 1) != grp) {
+              ++ir;
+              ++js;
+              continue;
+            }
             wait_raw(js);
             wait_slot();
             if (ok) conv_slab(raw + (js % kStg) * kStgBytes, ring + (ir % kStages) * kStageBytes, own);
@@ -1291,6 +1300,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
             ++js;
           }
           // k_pe: the two blocks' raw stages already hold the slot's boxes; copy them
+          if ((int)(ir & 1) != grp) {
+            ++ir;
+            js += 2;
+            return;
+          }
           wait_raw(js);
           wait_raw(js + 1);
           wait_slot();
@@ -1301,7 +1315,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
               const uint4* src = reinterpret_cast<const uint4*>(raw + ((js + b) % kStg) * kStgBytes);
               uint4* dst = reinterpret_cast<uint4*>(ring + (ir % kStages) * kStageBytes + b * kChunkBytes);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) dst[ct + kNumConvThreads * i] = src[ct + kNumConvThreads * i];
+              for (int i = 0; i < 8; ++i) dst[ct + kGrpThreads * i] = src[ct + kGrpThreads * i];
             }
           }
           if (!publish(js, 2)) return;
@@ -1311,6 +1325,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
           const int nb = blocks_in_tile(pc, t);
           for (int h = 0; h < 2; ++h) {
             for (int kb = 0; kb < nb; ++kb) {
+              if ((int)(ir & 1) != grp) {
+                ++ir;
+                ++js;
+                continue;
+              }
               wait_raw(js);
               wait_slot();
               if (ok) conv_vslab(raw + (js % kStg) * kStgBytes, ring + (ir % kStages) * kStageBytes);
