@@ -5,7 +5,7 @@
 //     lse = ln sum_s exp(lse_s),      out = sum_s exp(lse_s - lse) * O_s
 // (split-K merge; "DeepSeek speed test / FA3" article, section 2.1 names the split and
 // the softmax_lse side output).  HBM-bound: one warp per query row streams the S
-// partial rows with 16-byte loads and writes the bf16 row once.
+// partial rows with 16-byte loads, two splits in flight, and writes the bf16 row once.
 //
 // Grid (P, ceil(M / 8)): block x = p looks at partition p's first block; a split
 // sequence is exactly one whose cut opens a partition mid-sequence, and the first such
@@ -37,31 +37,53 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int part = blockIdx.x;
   if (part == 0) return;
+  // Three dependent round trips to memory: the partition's start, then every word of
+  // its sequence at once, then the partial lse values together with the first
+  // partial rows (the rest of the kernel is arithmetic on registers).
   const int b = meta[off_part_start() + 2 * part];
-  if (b >= B || meta[off_part_start() + 2 * part + 1] == 0) return;  // partition opens a sequence
-  if (meta[off_first_part(B) + b] + 1 != part) return;              // a later cut of the same sequence
+  const int k0 = meta[off_part_start() + 2 * part + 1];
+  if (b >= B || k0 == 0) return;  // partition opens a sequence (or is empty)
+  const int fp = meta[off_first_part(B) + b];
+  const int nblk = meta[off_nblk() + b];
+  const int ns = meta[off_num_splits(B) + b];
+  const int slot0 = meta[off_split_prefix(B) + b];
   const int n = seqlens[b];
+  const int ql = (q_lens != nullptr) ? q_lens[b] : s_q;
+  if (fp + 1 != part) return;  // a later cut of the same sequence
   // rows written as NaN already: invalid length, or a schedule built for another length
   if (n < 0 || (int64_t)n > (int64_t)max_blocks * kBlockSize) return;
-  if (meta[off_nblk() + b] != (n + kBlockSize - 1) / kBlockSize) return;
-  const int ql = q_lens ? q_lens[b] : s_q;
+  if (nblk != (n + kBlockSize - 1) / kBlockSize) return;
   if (ql < 0 || ql > s_q) return;  // invalid query count: NaN rows written already
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.y * kWarps + warp;
   if (row >= M) return;
   // a row tile holding only padding tokens had no pieces; its rows are written already
   if ((row / kRowsPerTile) * kRowsPerTile >= ql * (M / s_q)) return;
-  const int ns = meta[off_num_splits(B) + b];
-  uint2* orow = reinterpret_cast<uint2*>(out + ((int64_t)b * M + row) * kDLatent);
-  const int64_t slot0 = meta[off_split_prefix(B) + b];
-  // pass 1: max and sum over the partial lse values (every lane redundantly)
-  float m = -INFINITY;
-  bool any_nan = false;
-  for (int s = 0; s < ns; ++s) {
-    const float l = part_lse[(slot0 + s) * M + row];
+  const float* lse_row = part_lse + (int64_t)slot0 * M + row;  // split s at [s * M]
+  const float4* o_row = reinterpret_cast<const float4*>(part_o + ((int64_t)slot0 * M + row) * kDLatent) + lane;
+  const int64_t o_split = (int64_t)M * (kDLatent / 4);  // float4s between splits
+  constexpr int kGroup = 2;  // partial rows in flight per lane (64 registers)
+  float4 v[kGroup][4];
+  auto load_group = [&](int s0) {
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        v[j][k] = (s0 + j < ns) ? __ldg(o_row + (int64_t)(s0 + j) * o_split + 32 * k) : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  load_group(0);
+  // lse of split s is held by lane s % 32 (splits past 32 by further chunks)
+  const float l_lane = (lane < ns) ? __ldg(lse_row + (int64_t)lane * M) : -INFINITY;
+  float m = l_lane;
+  bool any_nan = (l_lane != l_lane);
+  for (int c = 32; c < ns; c += 32) {
+    const float l = (c + lane < ns) ? __ldg(lse_row + (int64_t)(c + lane) * M) : -INFINITY;
     any_nan |= (l != l);
     m = fmaxf(m, l);
   }
+  any_nan = __any_sync(0xffffffffu, any_nan);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   float res_lse;
   float4 acc[4];
 #pragma unroll
@@ -73,22 +95,34 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
   } else if (m == -INFINITY) {
     res_lse = -INFINITY;
   } else {
-    float z = 0.f;
-    for (int s = 0; s < ns; ++s) z += __expf(part_lse[(slot0 + s) * M + row] - m);
-    res_lse = m + __logf(z);
-    for (int s = 0; s < ns; ++s) {
-      const float w = __expf(part_lse[(slot0 + s) * M + row] - res_lse);
-      const float4* src = reinterpret_cast<const float4*>(part_o + ((slot0 + s) * M + row) * kDLatent);
+    // z = sum_s exp(lse_s - m), every lane's splits then a butterfly over the lanes
+    float z = (lane < ns) ? __expf(l_lane - m) : 0.f;
+    for (int c = 32; c < ns; c += 32)
+      if (c + lane < ns) z += __expf(__ldg(lse_row + (int64_t)(c + lane) * M) - m);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 v = src[k * 32 + lane];
-        acc[k].x += w * v.x;
-        acc[k].y += w * v.y;
-        acc[k].z += w * v.z;
-        acc[k].w += w * v.w;
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    res_lse = m + __logf(z);
+    // out = sum_s exp(lse_s - lse) O_s, accumulated in split order
+    for (int s0 = 0; s0 < ns; s0 += kGroup) {
+      if (s0 > 0) load_group(s0);
+#pragma unroll
+      for (int j = 0; j < kGroup; ++j) {
+        const int s = s0 + j;
+        if (s < ns) {  // warp-uniform
+          const float l = (s < 32) ? __shfl_sync(0xffffffffu, l_lane, s) : __ldg(lse_row + (int64_t)s * M);
+          const float w = __expf(l - res_lse);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            acc[k].x += w * v[j][k].x;
+            acc[k].y += w * v[j][k].y;
+            acc[k].z += w * v[j][k].z;
+            acc[k].w += w * v[j][k].w;
+          }
+        }
       }
     }
   }
+  uint2* orow = reinterpret_cast<uint2*>(out + ((int64_t)b * M + row) * kDLatent);
 #pragma unroll
   for (int k = 0; k < 4; ++k)
     orow[k * 32 + lane] = make_uint2(pack_bf16x2(acc[k].x, acc[k].y), pack_bf16x2(acc[k].z, acc[k].w));

@@ -52,8 +52,7 @@ constexpr int kNumProducers = 3;  // warps 0, 2, 3 (warp 0 also loads Q)
 constexpr int kMmaWarp = 1;
 constexpr int kSoftmaxWarp0 = 4;   // warps 4..11
 constexpr int kNumSoftmaxThreads = 256;
-constexpr int kConvWarp0 = 12;     // FP8 cache: warps 12..15
-constexpr int kNumConvThreads = 128;
+constexpr int kConvWarp0 = 12;     // FP8 cache: warps 12..15 (128 converter threads)
 constexpr int kMaxStages = 7;
 constexpr int kStageBytes = 16384;  // one bf16 ring slot
 constexpr int kChunkBytes = 8192;  // one 64-row x 64-column bf16 SW128 box
@@ -63,6 +62,9 @@ constexpr int kPBytes = 4 * kChunkBytes;  // 64 rows x 256 keys bf16
 constexpr int kSmemQ = 0;
 constexpr int kSmemP = kSmemQ + kQBytes;
 constexpr int kSmemRing = kSmemP + kPBytes;
+// The partition's last epilogue stages each of its (up to 4) rounds in its own 32 KB
+// from the start of shared memory: Q, P and the ring are contiguous and all idle then.
+constexpr int kEpiRoundBytes = 4 * kChunkBytes;
 // FP8 cache: raw stages of 8 KB (an e4m3 slab or one block of scaled k_pe) and two
 // buffers of per-key scales (4 blocks x 64 rows x 16 bytes, the scale in the first 4)
 constexpr int kStgBytes = 8192;
@@ -86,6 +88,7 @@ struct Cfg {
   static constexpr int kSmemScale = kSmemStg + kStg * kStgBytes;
   static constexpr int kSmemDyn = kSmemScale + (kFp8 ? 2 * kScaleBufBytes : 0);
   static_assert(kStages <= kMaxStages && kStg <= kMaxStg, "ring sizes");
+  static_assert(4 * kEpiRoundBytes <= kSmemStg, "the last epilogue's staging stays inside Q, P and the ring");
 };
 constexpr uint32_t kTmemO = 0, kTmemS0 = 256, kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only when the max grows by > 2^8
@@ -862,19 +865,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
       // inside the next piece's first tile (after that tile's weights are computed),
       // or after the last tile.  out = O / l (bf16) or the normalised fp32 partial,
       // written through TMA stores staged in the P buffer, which is free between a
-      // PV and the next P; then O's TMEM is handed back to the MMAs (o_free).
+      // PV and the next P; then O's TMEM is handed back to the MMAs (o_free).  After
+      // the partition's last tile (drain) the Q buffer and the ring are idle as well:
+      // each round then stages into its own 32 KB from the start of shared memory, and
+      // the stores of all rounds go out together after one barrier.
       bool pend = false, pend_direct = true;
       int pend_b = 0, pend_slot = 0;
       float pend_sc = 0.f, pend_lse = 0.f;
-      auto epilogue = [&]() {
+      auto epilogue = [&](bool drain) {
         const uint32_t to = tmem + kTmemO + 128 * g + lane_off;
         // per round every thread writes 128 bytes of its row (64 bf16 or 32 fp32 columns)
         // into box 2g + hk, laid out [64 rows][128 B] with the 128-byte swizzle, and one
         // thread stores the four boxes; rows past M are clipped by the tensor map
-        const uint32_t srow = sP + (2 * g + hk) * kChunkBytes + m * 128;
         const int rounds = pend_direct ? 2 : 4;
+        auto stage = [&](int r) -> uint32_t { return drain ? sQ + r * kEpiRoundBytes : sP; };
+        auto store_round = [&](int r) {
+#pragma unroll
+          for (int bx = 0; bx < 4; ++bx) {
+            const int gg = bx >> 1, hh = bx & 1;
+            if (pend_direct)
+              tma_store_3d(&p.tm_out, stage(r) + bx * kChunkBytes, 256 * gg + 128 * hh + 64 * r, y0, pend_b);
+            else
+              tma_store_3d(&p.tm_part, stage(r) + bx * kChunkBytes, 256 * gg + 128 * hh + 32 * r, y0, pend_slot);
+          }
+        };
 #pragma unroll 1
         for (int r = 0; r < rounds; ++r) {
+          const uint32_t srow = stage(r) + (2 * g + hk) * kChunkBytes + m * 128;
           uint32_t w[32];
           if (pend_direct) {
 #pragma unroll
@@ -893,13 +910,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
 #pragma unroll
             for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * pend_sc);
           }
-          if (r > 0) named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);  // previous round's boxes were read
+          if (r > 0 && !drain) named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);  // previous round's boxes were read
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(srow + ((q ^ (m & 7)) << 4)),
                          "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
                          : "memory");
           fence_proxy_async_smem();
+          if (drain) continue;
           if (r == 0) {
             go = named_bar_and(kBarSoftmax, kNumSoftmaxThreads, ok);
             if (!go) return;
@@ -907,16 +925,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
             named_bar_sync(kBarSoftmax, kNumSoftmaxThreads);
           }
           if (st == 0 && y0 < p.M) {  // a CTA whose 64 rows all lie past M stores nothing
-#pragma unroll
-            for (int bx = 0; bx < 4; ++bx) {
-              const int gg = bx >> 1, hh = bx & 1;
-              if (pend_direct)
-                tma_store_3d(&p.tm_out, sP + bx * kChunkBytes, 256 * gg + 128 * hh + 64 * r, y0, pend_b);
-              else
-                tma_store_3d(&p.tm_part, sP + bx * kChunkBytes, 256 * gg + 128 * hh + 32 * r, y0, pend_slot);
-            }
+            store_round(r);
             bulk_commit();
             bulk_wait_read_all();
+          }
+        }
+        if (drain) {
+          go = named_bar_and(kBarSoftmax, kNumSoftmaxThreads, ok);
+          if (!go) return;
+          if (st == 0 && y0 < p.M) {  // completion is awaited at teardown
+            for (int r = 0; r < rounds; ++r) store_round(r);
+            bulk_commit();
           }
         }
         if (row_valid && hk == 0 && g == 0) {
@@ -1097,7 +1116,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
             tc_fence_after();
             if (t == 0) {
               if (pend) {
-                epilogue();
+                epilogue(false);
                 if (!go) break;
               }
             } else if (__any_sync(0xffffffffu, rescale)) {
@@ -1197,7 +1216,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
         ok = wait_bar(&ctrl, p, smem_u32(&ctrl.p_free), pv_count & 1) && ok;
         ++pv_count;
         tc_fence_after();
-        epilogue();
+        epilogue(true);
       }
     }
     // =======================================================================
