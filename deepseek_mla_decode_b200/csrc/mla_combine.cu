@@ -5,9 +5,12 @@
 //     lse = ln sum_s exp(lse_s),      out = sum_s exp(lse_s - lse) * O_s
 // (split-K merge; "DeepSeek speed test / FA3" article, section 2.1 names the split and
 // the softmax_lse side output).  HBM-bound: one warp per query row streams the S
-// partial rows with 16-byte loads, two splits in flight, and writes the bf16 row once.
+// partial rows with 16-byte loads and writes the bf16 row once.  Batches of many
+// sequences (few splits each, many rows) take one warp per row with two splits in
+// flight; batches of few sequences (long ones, cut into many splits, few rows) take
+// four warps per row, each over 128 columns with eight splits in flight.
 //
-// Grid (P, ceil(M / 8)): block x = p looks at partition p's first block; a split
+// Grid (P, ceil(M * kColParts / 8)): block x = p looks at partition p's first block; a split
 // sequence is exactly one whose cut opens a partition mid-sequence, and the first such
 // partition (first_part + 1) owns its merge, so only blocks with work touch memory.
 // Rows of sequences that no partition covers (no visible key, invalid length, a block
@@ -23,12 +26,16 @@ namespace mla {
 namespace {
 
 constexpr int kWarps = 8;
+constexpr int kWideBatch = 16;  // batches below this many sequences take four warps per row
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// kColParts warps per query row, each over 512 / kColParts columns; kGroup partial rows
+// in flight per lane (both give 32 registers of loads)
+template <int kColParts, int kGroup>
 __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
     const int32_t* __restrict__ meta, const int32_t* __restrict__ seqlens, const int32_t* __restrict__ q_lens,
     int max_blocks, int B, int s_q, int M, const float* __restrict__ part_o, const float* __restrict__ part_lse,
@@ -55,20 +62,22 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
   if (nblk != (n + kBlockSize - 1) / kBlockSize) return;
   if (ql < 0 || ql > s_q) return;  // invalid query count: NaN rows written already
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.y * kWarps + warp;
+  const int wid = blockIdx.y * kWarps + warp;
+  const int row = wid / kColParts, part_col = wid % kColParts;
   if (row >= M) return;
   // a row tile holding only padding tokens had no pieces; its rows are written already
   if ((row / kRowsPerTile) * kRowsPerTile >= ql * (M / s_q)) return;
   const float* lse_row = part_lse + (int64_t)slot0 * M + row;  // split s at [s * M]
-  const float4* o_row = reinterpret_cast<const float4*>(part_o + ((int64_t)slot0 * M + row) * kDLatent) + lane;
+  constexpr int kF4 = 4 / kColParts;  // float4s per lane and split
+  const float4* o_row =
+      reinterpret_cast<const float4*>(part_o + ((int64_t)slot0 * M + row) * kDLatent) + part_col * 32 * kF4 + lane;
   const int64_t o_split = (int64_t)M * (kDLatent / 4);  // float4s between splits
-  constexpr int kGroup = 2;  // partial rows in flight per lane (64 registers)
-  float4 v[kGroup][4];
+  float4 v[kGroup][kF4];
   auto load_group = [&](int s0) {
 #pragma unroll
     for (int j = 0; j < kGroup; ++j)
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
+      for (int k = 0; k < kF4; ++k)
         v[j][k] = (s0 + j < ns) ? __ldg(o_row + (int64_t)(s0 + j) * o_split + 32 * k) : make_float4(0.f, 0.f, 0.f, 0.f);
   };
   load_group(0);
@@ -85,13 +94,13 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   float res_lse;
-  float4 acc[4];
+  float4 acc[kF4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = 0; k < kF4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (any_nan) {
     res_lse = __int_as_float(0x7fc00000);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) acc[k] = make_float4(res_lse, res_lse, res_lse, res_lse);
+    for (int k = 0; k < kF4; ++k) acc[k] = make_float4(res_lse, res_lse, res_lse, res_lse);
   } else if (m == -INFINITY) {
     res_lse = -INFINITY;
   } else {
@@ -112,7 +121,7 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
           const float l = (s < 32) ? __shfl_sync(0xffffffffu, l_lane, s) : __ldg(lse_row + (int64_t)s * M);
           const float w = __expf(l - res_lse);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int k = 0; k < kF4; ++k) {
             acc[k].x += w * v[j][k].x;
             acc[k].y += w * v[j][k].y;
             acc[k].z += w * v[j][k].z;
@@ -122,11 +131,11 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
       }
     }
   }
-  uint2* orow = reinterpret_cast<uint2*>(out + ((int64_t)b * M + row) * kDLatent);
+  uint2* orow = reinterpret_cast<uint2*>(out + ((int64_t)b * M + row) * kDLatent) + part_col * 32 * kF4;
 #pragma unroll
-  for (int k = 0; k < 4; ++k)
+  for (int k = 0; k < kF4; ++k)
     orow[k * 32 + lane] = make_uint2(pack_bf16x2(acc[k].x, acc[k].y), pack_bf16x2(acc[k].z, acc[k].w));
-  if (lane == 0) lse[(int64_t)b * M + row] = res_lse;
+  if (lane == 0 && part_col == 0) lse[(int64_t)b * M + row] = res_lse;
 }
 
 }  // namespace
@@ -134,8 +143,11 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
 cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, const int32_t* q_lens, int max_blocks,
                            int B, int s_q, int M, int P, const float* part_o, const float* part_lse, void* out, float* lse,
                            cudaStream_t stream) {
+  // few sequences: long ones with many splits and few rows to merge
+  const bool wide = B < kWideBatch;
+  const int parts = wide ? 4 : 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(P, (M + kWarps - 1) / kWarps);
+  cfg.gridDim = dim3(P, (M * parts + kWarps - 1) / kWarps);
   cfg.blockDim = dim3(kWarps * 32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -144,7 +156,10 @@ cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, const in
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, combine_kernel, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o, part_lse,
+  if (wide)
+    return cudaLaunchKernelEx(&cfg, combine_kernel<4, 8>, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o,
+                              part_lse, reinterpret_cast<__nv_bfloat16*>(out), lse);
+  return cudaLaunchKernelEx(&cfg, combine_kernel<1, 2>, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o, part_lse,
                             reinterpret_cast<__nv_bfloat16*>(out), lse);
 }
 
