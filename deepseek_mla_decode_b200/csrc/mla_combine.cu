@@ -4,13 +4,13 @@
 // divided by its own softmax sum) and their log-sum-exps lse_s.  The exact merge is
 //     lse = ln sum_s exp(lse_s),      out = sum_s exp(lse_s - lse) * O_s
 // (split-K merge; "DeepSeek speed test / FA3" article, section 2.1 names the split and
-// the softmax_lse side output).  HBM-bound: one warp per query row streams the S
-// partial rows with 16-byte loads and writes the bf16 row once.  Batches of many
+// the softmax_lse side output).  HBM-bound: the warps of a query row stream its S
+// partial rows with 16-byte loads and write the bf16 row once.  Batches of many
 // sequences (few splits each, many rows) take one warp per row with two splits in
 // flight; batches of few sequences (long ones, cut into many splits, few rows) take
 // four warps per row, each over 128 columns with eight splits in flight.
 //
-// Grid (P, ceil(M * kColParts / 8)): block x = p looks at partition p's first block; a split
+// Grid (P, ceil(M * c / 8)), c warps per row: block x = p looks at partition p's first block; a split
 // sequence is exactly one whose cut opens a partition mid-sequence, and the first such
 // partition (first_part + 1) owns its merge, so only blocks with work touch memory.
 // Rows of sequences that no partition covers (no visible key, invalid length, a block

@@ -17,8 +17,10 @@
 // longest rows first.  Warp 0 issues the TMA loads (both tiles' Q once; per key block
 // its K slab, V slab and the keys' scales, shared by the two tiles), warp 1 the MMAs,
 // warps 4..7 the softmax of tile 0 and warps 8..11 that of tile 1 (one thread per
-// query row = TMEM lane).  The MMA order QK(0, j+1), PV(1, j), QK(1, j+1), PV(0, j+1)
-// ... lets one tile's softmax run while the tensor core works on the other tile.
+// query row = TMEM lane).  Per key block j the MMA warp issues QK(0, j+1), QK(1, j+1),
+// PV(0, j), PV(1, j): the next block's scores need only this block's scores read out
+// of TMEM, so they are computed while both tiles' softmax works on block j, and each
+// tile's softmax waits for the tensor core only briefly between blocks.
 // TMEM: S of tile t in columns [128 t, 128 t + 128), O of tile t in [256 + 128 t, ...).
 // Every wait is bounded: a timeout sets MLA_DEVICE_ERR_TIMEOUT, every role stops at its
 // next wait, the CTA drains its tensor-core work and returns.
@@ -283,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
     }
   } else if (warp == kMmaWarp) {
     // =====================================================================
-    // MMA issuer: QK(0, 0), QK(1, 0), then per key block j: PV(0, j), QK(0, j + 1),
-    // PV(1, j), QK(1, j + 1), and the block's stage is released
+    // MMA issuer: QK(0, 0), QK(1, 0), then per key block j: QK(0, j + 1), QK(1, j + 1),
+    // PV(0, j), PV(1, j), and the block's stage is released
     // =====================================================================
     regs_dec<kRegsIssue>();
     bool ok = wait_bar(&ctrl, p, smem_u32(&ctrl.q_full), 0);
@@ -331,14 +333,14 @@ __global__ void __launch_bounds__(kThreads, 1) sage_attn_kernel(const __grid_con
     qk(0, 0);
     if (nk1 > 0) qk(1, 0);
     for (int j = 0; j < nkb && ok; ++j) {
+      // S of block j+1 needs only S of block j read out (s_free, right after the
+      // softmax's TMEM load), so it is computed while the softmax works on block j
 #pragma unroll
-      for (int t = 0; t < kTiles; ++t) {
-        const int nkt = t == 0 ? nk0 : nk1;
-        if (j < nkt) {
-          pv(t, j);
-          if (j + 1 < nkt) qk(t, j + 1);
-        }
-      }
+      for (int t = 0; t < kTiles; ++t)
+        if (j + 1 < (t == 0 ? nk0 : nk1)) qk(t, j + 1);
+#pragma unroll
+      for (int t = 0; t < kTiles; ++t)
+        if (j < (t == 0 ? nk0 : nk1)) pv(t, j);
       if (ok && elected) commit(smem_u32(&ctrl.empty[j % kStages]));  // after both tiles' PV of block j
       __syncwarp();
     }
