@@ -13,6 +13,7 @@
 //   sq, sk fp32 [H][S_pad]         sv fp32 [H][128]       vmax uint32 [H][128]
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <algorithm>
 #include <cstdint>
 #include "sage_internal.h"
 
@@ -20,57 +21,92 @@ namespace mla {
 namespace sage {
 namespace {
 
-// One warp per (token, head) row of 192 bf16: lanes 0..23 hold 8 values each.
+// Q / K rows: a warp quantises four (token, head) rows of 192 bf16 at a time, eight
+// lanes per row, 24 values (three 16-byte loads) per lane; grid-stride over the rows.
+constexpr int kRowLanes = 8, kRowVals = kDQK / kRowLanes;  // 24
 __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int8_t* __restrict__ q8,
                                                         float* __restrict__ scale, int S, int S_pad, int H) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);  // = token * H + head over S_pad tokens
-  if (row >= (int64_t)S_pad * H) return;
-  const int t = (int)(row / H), h = (int)(row % H);
-  float v[8];
-  bool live = lane < kDQK / 8 && t < S;
-  if (live) {
-    const uint4 w = reinterpret_cast<const uint4*>(x + ((int64_t)t * H + h) * kDQK)[lane];
+  const int lane = threadIdx.x & 31, sub = lane & (kRowLanes - 1);
+  const int64_t nrows = (int64_t)S_pad * H;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t row = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4 + (lane >> 3); ;
+       row += warps * 4) {
+    // the warp's four rows advance together; lanes past the last row idle but stay in
+    // the shuffles
+    const int64_t row0 = row - (lane >> 3);
+    if (row0 >= nrows) break;
+    const bool have = row < nrows;
+    const int t = have ? (int)(row / H) : 0, h = have ? (int)(row % H) : 0;
+    float v[kRowVals];
+    if (have && t < S) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + ((int64_t)t * H + h) * kDQK + sub * kRowVals);
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        const uint4 w = src[k];
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[8 * k + 2 * i] = __uint_as_float(u[i] << 16);
+          v[8 * k + 2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < kRowVals; ++i) v[i] = 0.f;
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < kRowVals; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+    for (int o = kRowLanes / 2; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = __fdiv_rn(amax, 127.0f);
+    uint32_t packed[kRowVals / 4] = {0u, 0u, 0u, 0u, 0u, 0u};
+    if (s > 0.f) {
+#pragma unroll
+      for (int i = 0; i < kRowVals; ++i) {
+        int c = __float2int_rn(__fdiv_rn(v[i], s));
+        c = max(-127, min(127, c));
+        packed[i >> 2] |= (uint32_t)(c & 0xff) << (8 * (i & 3));
+      }
+    }
+    if (have) {
+      uint2* dst = reinterpret_cast<uint2*>(q8 + ((int64_t)h * S_pad + t) * kDQK + sub * kRowVals);
+#pragma unroll
+      for (int k = 0; k < 3; ++k) dst[k] = make_uint2(packed[2 * k], packed[2 * k + 1]);
+      if (sub == 0) scale[(int64_t)h * S_pad + t] = s;
+    }
+  }
+}
+
+// Channel maxima of V: block (token chunk, head); thread = (token row of 16, group of
+// 8 channels), 16-byte loads; the block reduces its maxima in shared memory, then one
+// integer atomicMax per channel (the maxima of non-negative floats order like their
+// bit patterns).
+constexpr int kVChunk = 256;
+__global__ void __launch_bounds__(256) vmax_kernel(const __nv_bfloat16* __restrict__ v, uint32_t* __restrict__ vmax,
+                                                   int S, int H) {
+  __shared__ float red[16][kDV];
+  const int h = blockIdx.y, g = threadIdx.x & 15, tr = threadIdx.x >> 4;  // channels 8 g .. 8 g + 7
+  const int t0 = blockIdx.x * kVChunk, t1 = min(S, t0 + kVChunk);
+  float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int t = t0 + tr; t < t1; t += 16) {
+    const uint4 w = reinterpret_cast<const uint4*>(v + ((int64_t)t * H + h) * kDV)[g];
     const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __uint_as_float(u[i] << 16);
-      v[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = 0.f;
-  }
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float s = __fdiv_rn(amax, 127.0f);
-  uint32_t packed[2] = {0u, 0u};
-  if (s > 0.f) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      int c = __float2int_rn(__fdiv_rn(v[i], s));
-      c = max(-127, min(127, c));
-      packed[i >> 2] |= (uint32_t)(c & 0xff) << (8 * (i & 3));
+      m[2 * i] = fmaxf(m[2 * i], fabsf(__uint_as_float(u[i] << 16)));
+      m[2 * i + 1] = fmaxf(m[2 * i + 1], fabsf(__uint_as_float(u[i] & 0xffff0000u)));
     }
   }
-  int8_t* dst = q8 + ((int64_t)h * S_pad + t) * kDQK;
-  if (lane < kDQK / 8) reinterpret_cast<uint2*>(dst)[lane] = make_uint2(packed[0], packed[1]);
-  if (lane == 0) scale[(int64_t)h * S_pad + t] = s;
-}
-
-// Channel maxima of V: block (token chunk, head), thread = channel; the maxima of
-// non-negative floats order like their bit patterns, so an integer atomicMax suffices.
-constexpr int kVChunk = 256;
-__global__ void __launch_bounds__(kDV) vmax_kernel(const __nv_bfloat16* __restrict__ v, uint32_t* __restrict__ vmax,
-                                                   int S, int H) {
-  const int h = blockIdx.y, d = threadIdx.x;
-  const int t0 = blockIdx.x * kVChunk, t1 = min(S, t0 + kVChunk);
-  float m = 0.f;
-  for (int t = t0; t < t1; ++t) m = fmaxf(m, fabsf(__bfloat162float(v[((int64_t)t * H + h) * kDV + d])));
-  atomicMax(vmax + h * kDV + d, __float_as_uint(m));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) red[tr][8 * g + i] = m[i];
+  __syncthreads();
+  if (threadIdx.x < kDV) {
+    float r = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) r = fmaxf(r, red[k][threadIdx.x]);
+    atomicMax(vmax + h * kDV + threadIdx.x, __float_as_uint(r));
+  }
 }
 
 __device__ __forceinline__ uint32_t e4m3x2_rn(float lo, float hi) {
@@ -80,31 +116,43 @@ __device__ __forceinline__ uint32_t e4m3x2_rn(float lo, float hi) {
 }
 
 // V codes, transposed through shared memory: block (64-token chunk, head) reads 64
-// tokens x 128 channels and writes 128 channel rows of 64 codes.
+// tokens x 128 channels with 16-byte loads (thread = token row of 16, group of 8
+// channels, four passes) and writes 128 channel rows of 64 codes.
 constexpr int kVtTokens = 64;
 __global__ void __launch_bounds__(256) vquant_kernel(const __nv_bfloat16* __restrict__ v,
                                                      const uint32_t* __restrict__ vmax, uint8_t* __restrict__ vt8,
                                                      float* __restrict__ sv, int S, int S_pad, int H) {
   __shared__ uint8_t tile[kDV][kVtTokens + 4];
   const int h = blockIdx.y, t0 = blockIdx.x * kVtTokens;
-  // each thread: one channel pair for 16 tokens
-  const int dp = threadIdx.x & 63;       // channel pair (2 dp, 2 dp + 1)
-  const int tq = threadIdx.x >> 6;       // token quarter
-  const float s0 = __fdiv_rn(__uint_as_float(vmax[h * kDV + 2 * dp]), 448.0f);
-  const float s1 = __fdiv_rn(__uint_as_float(vmax[h * kDV + 2 * dp + 1]), 448.0f);
-  for (int i = 0; i < kVtTokens / 4; ++i) {
-    const int tl = tq * (kVtTokens / 4) + i, t = t0 + tl;
-    uint32_t c = 0;
+  const int g = threadIdx.x & 15, tr = threadIdx.x >> 4;  // channels 8 g .. 8 g + 7; token row tr of 16
+  float sc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sc[i] = __fdiv_rn(__uint_as_float(vmax[h * kDV + 8 * g + i]), 448.0f);
+#pragma unroll
+  for (int pass = 0; pass < kVtTokens / 16; ++pass) {
+    const int tl = pass * 16 + tr, t = t0 + tl;
+    float x[8];
     if (t < S) {
-      const __nv_bfloat162 w = reinterpret_cast<const __nv_bfloat162*>(v + ((int64_t)t * H + h) * kDV)[dp];
-      const float a = s0 > 0.f ? __fdiv_rn(__low2float(w), s0) : 0.f;
-      const float b = s1 > 0.f ? __fdiv_rn(__high2float(w), s1) : 0.f;
-      c = e4m3x2_rn(a, b);
-      if (!(s0 > 0.f)) c &= 0xff00u;
-      if (!(s1 > 0.f)) c &= 0x00ffu;
+      const uint4 w = reinterpret_cast<const uint4*>(v + ((int64_t)t * H + h) * kDV)[g];
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(u[i] << 16);
+        x[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = 0.f;
     }
-    tile[2 * dp][tl] = (uint8_t)(c & 0xff);
-    tile[2 * dp + 1][tl] = (uint8_t)(c >> 8);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const bool l0 = sc[i] > 0.f && t < S, l1 = sc[i + 1] > 0.f && t < S;
+      uint32_t c = e4m3x2_rn(l0 ? __fdiv_rn(x[i], sc[i]) : 0.f, l1 ? __fdiv_rn(x[i + 1], sc[i + 1]) : 0.f);
+      if (!l0) c &= 0xff00u;
+      if (!l1) c &= 0x00ffu;
+      tile[8 * g + i][tl] = (uint8_t)(c & 0xff);
+      tile[8 * g + i + 1][tl] = (uint8_t)(c >> 8);
+    }
   }
   __syncthreads();
   // 128 rows x 64 bytes out: thread -> (row, 16-byte quarter); two rows per pass
@@ -118,11 +166,9 @@ __global__ void __launch_bounds__(256) vquant_kernel(const __nv_bfloat16* __rest
     }
     reinterpret_cast<uint4*>(vt8 + ((int64_t)h * kDV + r) * S_pad + t0)[qd] = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  if (blockIdx.x == 0) {
-    if (tq == 0) {
-      sv[h * kDV + 2 * dp] = s0;
-      sv[h * kDV + 2 * dp + 1] = s1;
-    }
+  if (blockIdx.x == 0 && tr == 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sv[h * kDV + 8 * g + i] = sc[i];
   }
 }
 
@@ -132,12 +178,13 @@ cudaError_t launch_quantize(const void* q, const void* k, const void* v, int S, 
                             cudaStream_t stream) {
   const int S_pad = padded_len(S);
   const int64_t rows = (int64_t)S_pad * H;
-  const unsigned grid_rows = (unsigned)((rows + 7) / 8);
+  // 32 rows per block of 8 warps, at most 16 blocks per SM's worth (grid-stride beyond)
+  const unsigned grid_rows = (unsigned)std::min<int64_t>((rows + 31) / 32, 148 * 16);
   quant_rows_kernel<<<grid_rows, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q), ws.q8, ws.sq, S, S_pad, H);
   quant_rows_kernel<<<grid_rows, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), ws.k8, ws.sk, S, S_pad, H);
   cudaError_t e = cudaMemsetAsync(ws.vmax, 0, (size_t)H * kDV * sizeof(uint32_t), stream);
   if (e != cudaSuccess) return e;
-  vmax_kernel<<<dim3((S + kVChunk - 1) / kVChunk, H), kDV, 0, stream>>>(static_cast<const __nv_bfloat16*>(v),
+  vmax_kernel<<<dim3((S + kVChunk - 1) / kVChunk, H), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(v),
                                                                           ws.vmax, S, H);
   vquant_kernel<<<dim3(S_pad / kVtTokens, H), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(v), ws.vmax,
                                                                  ws.vt8, ws.sv, S, S_pad, H);
