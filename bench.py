@@ -116,6 +116,52 @@ def bench_prefill(mla, dev, steps, warmup, S=None, H=None):
             "tokens_per_s": S / ((att_ms + quant_ms) * 1e-3), "steps": steps}
 
 
+def bench_absorb(mla, dev, steps, warmup, flush, B=256, s_q=1, H=128):
+    """The absorption GEMMs either side of the decode at the serving shape: q_nope =
+    W_UK^T q_heads and y = W_UV o per head, on seeded device inputs (N(0, 1) rows, N(0,
+    0.05^2) weights), each call timed with CUDA events after an L2 flush.  Memory-bound:
+    the algorithmic bytes are the rows read and written plus the head weights."""
+    import torch
+
+    R = B * s_q
+    g = torch.Generator(device=dev).manual_seed(4242)
+    q_heads = torch.randn((B, s_q, H, 128), generator=g, device=dev).to(torch.bfloat16)
+    o_lat = torch.randn((B, s_q, H, 512), generator=g, device=dev).to(torch.bfloat16)
+    w_uk = (0.05 * torch.randn((H, 128, 512), generator=g, device=dev)).to(torch.bfloat16)
+    w_uv = (0.05 * torch.randn((H, 128, 512), generator=g, device=dev)).to(torch.bfloat16)
+    q_nope = torch.empty((B, s_q, H, 512), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((B, s_q, H, 128), dtype=torch.bfloat16, device=dev)
+    st = torch.cuda.current_stream()
+    for _ in range(warmup):
+        mla.absorb_q(q_heads, w_uk, q_nope=q_nope, stream=st)
+        mla.absorb_out(o_lat, w_uv, y=y, stream=st)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for e in ev:
+        flush()
+        e[0].record(st)
+        mla.absorb_q(q_heads, w_uk, q_nope=q_nope, stream=st)
+        e[1].record(st)
+        flush()
+        e[2].record(st)
+        mla.absorb_out(o_lat, w_uv, y=y, stream=st)
+        e[3].record(st)
+    torch.cuda.synchronize()
+    hbm, _, _, src = load_peaks()
+    wbytes = H * 128 * 512 * 2
+    res = {}
+    for name, i0, nbytes in (("absorb_q", 0, R * H * (128 + 512) * 2 + wbytes),
+                             ("absorb_out", 2, R * H * (512 + 128) * 2 + wbytes)):
+        ms = sum(e[i0].elapsed_time(e[i0 + 1]) for e in ev) / steps
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[f"{name}_b{B}"] = {
+            "workload": f"{name} B={B}, s_q={s_q}, H={H} (bf16, fp32 accumulation)",
+            "kernel": f"absorb_kernel ({name})",
+            "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+            "peak_source": f"{src} HBM copy", "kernel_avg_us": ms * 1e3, "roofline_us": nbytes / (hbm * 1e9) * 1e6,
+            "algorithmic_bytes": nbytes, "flops": 2 * R * H * 128 * 512, "steps": steps}
+    return res
+
+
 def metric_name(w):
     """The metric string both arms print, so their lines can be divided."""
     return f"MLA decode TFLOP/s ({w.name}: B={w.B}, s_q={w.s_q}, H={w.H})"
@@ -462,6 +508,8 @@ def main():
     ap.add_argument("--prefill-steps", type=int, default=5,
                     help="timed runs of the quantised 64K-token prefill (0 = skip)")
     ap.add_argument("--prefill-shape", default="65536,16", help="S,H of the quantised prefill")
+    ap.add_argument("--absorb-steps", type=int, default=30,
+                    help="timed calls of each absorption GEMM at the serving shape (0 = skip)")
     ap.add_argument("--kv-format", default="bf16", choices=["bf16", "fp8"],
                     help="cache of the headline run: bf16 rows, or the packed FP8 rows (quantised once, untimed)")
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -597,6 +645,10 @@ def main():
             per_workload[name + "_fp8"] = roofline(wi, ti, args.per_workload_steps, fp8=True)
             del ri
             torch.cuda.empty_cache()
+
+    if world == 1 and args.absorb_steps > 0:
+        per_workload.update(bench_absorb(mla, dev, args.absorb_steps, args.warmup, flusher))
+        torch.cuda.empty_cache()
 
     if world == 1 and args.prefill_steps > 0:
         pS, pH = (int(x) for x in args.prefill_shape.split(","))

@@ -8,12 +8,16 @@
 // for every query row r (= b * s_q + i) and head h.  Both are batched GEMMs over the
 // heads: rows [R, 128] x [128, 512] per head, and rows [R, 512] x [512, 128].
 //
-// One CTA (128 threads) computes 128 rows of one head: TMA loads the row tile and
-// the head's weight into shared memory (128-byte swizzle), one thread issues 1-CTA
-// tcgen05 MMAs (M = 128) into a TMEM accumulator, and the four warps move their 32
-// TMEM lanes (rows) out through a swizzled staging tile and TMA stores.  Memory-bound:
-// the weights (16.8 MB per projection for 128 heads) and the rows are read once per
-// row tile; rows past R are zero-filled on load and clipped on store.
+// One CTA (128 threads) computes 128 rows x 128 output columns of one head: TMA loads
+// the row tile and the head's weight slice into shared memory (128-byte swizzle), one
+// thread issues 1-CTA tcgen05 MMAs (M = 128, N = 128) into a TMEM accumulator, and the
+// four warps move their 32 TMEM lanes (rows) out through a swizzled staging tile and
+// TMA stores.  The q side's 512 output columns are four CTAs; the out side's 512-deep
+// contraction runs in four phases of 128.  Each CTA holds 64 KB of shared memory, so
+// three share an SM and one's loads overlap another's MMAs and stores.  Memory-bound:
+// the weights (16.8 MB per projection for 128 heads) are read once from HBM, the rows
+// once per row tile and column slice (L2 serves the repeats); rows past R are
+// zero-filled on load and clipped on store.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -80,10 +84,11 @@ __device__ __forceinline__ void wait_bounded(uint32_t bar, uint32_t parity) {
   }
 }
 
-// N output columns, K contraction, weights MN-major (q side: W_UK[h] is [k][n]) or
-// K-major (out side: W_UV[h] is [n][k]); the contraction runs in phases of KP.
+// N output columns per CTA (slice blockIdx.z of the projection's), K contraction,
+// weights MN-major (q side: W_UK[h] is [k][n]) or K-major (out side: W_UV[h] is
+// [n][k]); the contraction runs in phases of KP.
 template <int N, int K, bool B_MN, int KP>
-__global__ void __launch_bounds__(kAbThreads, 1) absorb_kernel(const __grid_constant__ AbsorbParams p) {
+__global__ void __launch_bounds__(kAbThreads) absorb_kernel(const __grid_constant__ AbsorbParams p) {
   static_assert(K % KP == 0 && KP % 64 == 0 && N % 64 == 0, "tile shape");
   constexpr int kKB = KP / 64;                                   // 64-wide k blocks per phase
   constexpr int kABytes = kKB * 2 * kBox;                        // 128 rows x KP
@@ -92,16 +97,17 @@ __global__ void __launch_bounds__(kAbThreads, 1) absorb_kernel(const __grid_cons
   constexpr uint32_t kIdesc = make_idesc_bf16(128, kNMma, false, B_MN);
   constexpr uint32_t kCols = N < 32 ? 32 : N;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_load, bar_mma;
+  __shared__ __align__(8) uint64_t bar_load, bar_mma, bar_done;
   __shared__ uint32_t tmem_base;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sA = smem_u32(smem), sB = sA + kABytes;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int h = blockIdx.y, r0 = blockIdx.x * kRowTile;
+  const int h = blockIdx.y, r0 = blockIdx.x * kRowTile, n0 = blockIdx.z * N;
 
   if (tid == 0) {
     mbar_init(smem_u32(&bar_load), 1);
     mbar_init(smem_u32(&bar_mma), 1);
+    mbar_init(smem_u32(&bar_done), 1);
     fence_mbar_init();
     prefetch_tmap(&p.tm_a);
     prefetch_tmap(&p.tm_b);
@@ -127,9 +133,10 @@ __global__ void __launch_bounds__(kAbThreads, 1) absorb_kernel(const __grid_cons
         const int k0 = ph * KP + 64 * i;
         tma_load_3d(sA + i * 2 * kBox, &p.tm_a, bl, k0, h, r0);
         if (B_MN) {
-          for (int j = 0; j < N / 64; ++j) tma_load_3d(sB + (i * (N / 64) + j) * kBox, &p.tm_b, bl, 64 * j, k0, h);
+          for (int j = 0; j < N / 64; ++j)
+            tma_load_3d(sB + (i * (N / 64) + j) * kBox, &p.tm_b, bl, n0 + 64 * j, k0, h);
         } else {
-          tma_load_3d(sB + i * (N / 64) * kBox, &p.tm_b, bl, k0, 0, h);
+          tma_load_3d(sB + i * (N / 64) * kBox, &p.tm_b, bl, k0, n0, h);
         }
       }
       wait_bounded(bl, ph & 1);
@@ -152,10 +159,11 @@ __global__ void __launch_bounds__(kAbThreads, 1) absorb_kernel(const __grid_cons
       }
       commit_1sm(bm);
     }
+    commit_1sm(smem_u32(&bar_done));  // completes once every MMA above has
   }
-  // every thread waits for the last phase's MMAs (phase by phase: a parity wait only
-  // tells completed from in-progress for the phase right after the last completed one)
-  for (int ph = 0; ph < K / KP; ++ph) wait_bounded(smem_u32(&bar_mma), ph & 1);
+  // every thread waits for all MMAs on a barrier with a single phase (a parity wait on
+  // bar_mma, which completes once per phase, could alias a later phase)
+  wait_bounded(smem_u32(&bar_done), 0);
   tc_fence_after();
 
   // epilogue: warp w owns TMEM lanes (rows) 32w..32w+31; column block j of 64 goes to
@@ -184,7 +192,7 @@ __global__ void __launch_bounds__(kAbThreads, 1) absorb_kernel(const __grid_cons
   tc_fence_before();
   __syncthreads();
   if (tid == 0) {
-    for (int j = 0; j < N / 64; ++j) tma_store_3d(&p.tm_c, sA + j * 2 * kBox, 64 * j, h, r0);
+    for (int j = 0; j < N / 64; ++j) tma_store_3d(&p.tm_c, sA + j * 2 * kBox, n0 + 64 * j, h, r0);
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
@@ -201,8 +209,11 @@ constexpr int absorb_smem() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int N, int K, bool B_MN, int KP>
+// NT output columns in all, N per CTA
+template <int NT, int N, int K, bool B_MN, int KP>
 mla_status_t launch_absorb(const void* rows, const void* w, void* outp, int R, int H, cudaStream_t stream) {
+  static_assert(NT % N == 0, "column slices");
+  static_assert(2 * (KP / 64) * kBox >= (N / 64) * 2 * kBox, "the epilogue stages the output in the row tile's space");
   if (!rows || !w || !outp) return MLA_ERR_INVALID_ARG;
   if (R < 1 || H < 1 || H > 65535) return MLA_ERR_INVALID_ARG;
   if (!aligned16(rows) || !aligned16(w) || !aligned16(outp)) return MLA_ERR_INVALID_ARG;
@@ -217,19 +228,19 @@ mla_status_t launch_absorb(const void* rows, const void* w, void* outp, int R, i
     if (!encode_tiled_bf16(&prm.tm_a, rows, 3, dims, strides, box)) return MLA_ERR_INVALID_ARG;
   }
   if (B_MN) {  // W[h] is [k = 128][n = 512]
-    const cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)K, (cuuint64_t)H};
-    const cuuint64_t strides[2] = {(cuuint64_t)N * 2, (cuuint64_t)K * N * 2};
+    const cuuint64_t dims[3] = {(cuuint64_t)NT, (cuuint64_t)K, (cuuint64_t)H};
+    const cuuint64_t strides[2] = {(cuuint64_t)NT * 2, (cuuint64_t)K * NT * 2};
     const cuuint32_t box[3] = {64, 64, 1};
     if (!encode_tiled_bf16(&prm.tm_b, w, 3, dims, strides, box)) return MLA_ERR_INVALID_ARG;
   } else {  // W[h] is [n = 128][k = 512]
-    const cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)N, (cuuint64_t)H};
-    const cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)N * K * 2};
+    const cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)NT, (cuuint64_t)H};
+    const cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)NT * K * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)N, 1};
     if (!encode_tiled_bf16(&prm.tm_b, w, 3, dims, strides, box)) return MLA_ERR_INVALID_ARG;
   }
   {
-    const cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)R};
-    const cuuint64_t strides[2] = {(cuuint64_t)N * 2, (cuuint64_t)H * N * 2};
+    const cuuint64_t dims[3] = {(cuuint64_t)NT, (cuuint64_t)H, (cuuint64_t)R};
+    const cuuint64_t strides[2] = {(cuuint64_t)NT * 2, (cuuint64_t)H * NT * 2};
     const cuuint32_t box[3] = {64, 1, kRowTile};
     if (!encode_tiled_bf16(&prm.tm_c, outp, 3, dims, strides, box)) return MLA_ERR_INVALID_ARG;
   }
@@ -237,7 +248,7 @@ mla_status_t launch_absorb(const void* rows, const void* w, void* outp, int R, i
   auto kern = absorb_kernel<N, K, B_MN, KP>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return MLA_ERR_CUDA;
-  dim3 grid((R + kRowTile - 1) / kRowTile, H);
+  dim3 grid((R + kRowTile - 1) / kRowTile, H, NT / N);
   kern<<<grid, kAbThreads, smem, stream>>>(prm);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
@@ -247,10 +258,11 @@ mla_status_t launch_absorb(const void* rows, const void* w, void* outp, int R, i
 
 extern "C" mla_status_t mla_absorb_q(const void* q_heads, const void* w_uk, void* q_nope, int R, int H,
                                      void* stream) {
-  return mla::launch_absorb<512, 128, true, 128>(q_heads, w_uk, q_nope, R, H, static_cast<cudaStream_t>(stream));
+  return mla::launch_absorb<512, 128, 128, true, 128>(q_heads, w_uk, q_nope, R, H,
+                                                      static_cast<cudaStream_t>(stream));
 }
 
 extern "C" mla_status_t mla_absorb_out(const void* o_latent, const void* w_uv, void* y, int R, int H,
                                        void* stream) {
-  return mla::launch_absorb<128, 512, false, 256>(o_latent, w_uv, y, R, H, static_cast<cudaStream_t>(stream));
+  return mla::launch_absorb<128, 128, 512, false, 128>(o_latent, w_uv, y, R, H, static_cast<cudaStream_t>(stream));
 }
