@@ -63,6 +63,81 @@ def algorithmic_work(seqlens, s_q, H, causal, row_bytes=D_QK * 2):
     return flops, cache_bytes, cache_bytes + q_bytes + out_bytes
 
 
+def ragged_work(seqlens, q_lens, H, causal, row_bytes=D_QK * 2):
+    """algorithmic_work with q_lens[b] query tokens for sequence b (the last q_lens[b]
+    cache positions): FLOPs over each token's visible keys, the cache rows of every
+    sequence with at least one token once, q / out / lse of the tokens."""
+    flops = 0
+    keys = 0
+    tokens = 0
+    for n, ql in zip(np.asarray(seqlens).tolist(), np.asarray(q_lens).tolist()):
+        if ql <= 0:
+            continue
+        keys += max(int(n), 0)
+        tokens += ql
+        for i in range(ql):
+            vis = n if not causal else max(0, min(n, n - ql + i + 1))
+            flops += max(vis, 0) * H * 2 * (D_QK + D_LATENT)
+    cache_bytes = keys * row_bytes
+    io_bytes = tokens * H * (D_QK * 2 + D_LATENT * 2 + 4)
+    return flops, cache_bytes, cache_bytes + io_bytes
+
+
+def bench_ragged(mla, dev, steps, warmup, flush, B=128, s_q=4, H=128, seed=1005):
+    """Speculative-decoding verification with per-sequence accepted drafts: B = 128
+    sequences, up to s_q = 4 query tokens each with q_lens[b] drawn uniformly from
+    1..4, causal, lengths U[1024, 8192] as in the MTP workload.  Times the public
+    mla_decode_ragged call (attention and LSE combine) after an L2 flush; the roofline
+    is the slower of the cache bytes at HBM bandwidth and the FLOPs at the bf16 peak."""
+    import torch
+    from deepseek_mla_decode_b200.workloads import make_inputs
+
+    rng = np.random.default_rng(seed + 7919)
+    seqlens = rng.integers(1024, 8192 + 1, size=B, dtype=np.int64).astype(np.int32)
+    q_lens = rng.integers(1, s_q + 1, size=B, dtype=np.int64).astype(np.int32)
+    inp = make_inputs(B, s_q, H, seqlens, seed, causal=True)
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q_nope, q_pe, kv = bf16(inp.q_nope), bf16(inp.q_pe), bf16(inp.kv_cache)
+    table = torch.from_numpy(inp.block_table).to(dev)
+    lens = torch.from_numpy(inp.cache_seqlens).to(dev)
+    qls = torch.from_numpy(q_lens).to(dev)
+    st = torch.cuda.current_stream()
+    meta = mla.get_metadata(lens, s_q, H, stream=st)
+    ws = torch.empty(mla.workspace_size(B, s_q, H), dtype=torch.uint8, device=dev)
+    out = torch.empty((B, s_q, H, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, s_q, H), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(warmup):
+        mla.decode_ragged(q_nope, q_pe, kv, table, lens, qls, inp.softmax_scale, True, meta, workspace=ws, out=out,
+                          lse=lse, status=status, stream=st)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    for e in ev:
+        flush()
+        e[0].record(st)
+        mla.decode_ragged(q_nope, q_pe, kv, table, lens, qls, inp.softmax_scale, True, meta, workspace=ws, out=out,
+                          lse=lse, status=status, stream=st)
+        e[1].record(st)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} in the ragged decode")
+    ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+    hbm, tc, _, src = load_peaks()
+    flops, cache_bytes, _ = ragged_work(seqlens, q_lens, H, True)
+    t_hbm, t_tc = cache_bytes / (hbm * 1e9), flops / (tc * 1e12)
+    bound = "tensor" if t_tc >= t_hbm else "hbm"
+    roof = max(t_hbm, t_tc)
+    achieved = flops / (ms * 1e-3) / 1e12 if bound == "tensor" else cache_bytes / (ms * 1e-3) / 1e9
+    return {"workload": f"ragged MTP verification B={B}, s_q<={s_q} (q_lens U[1, {s_q}], mean "
+                        f"{float(q_lens.mean()):.2f}), H={H}, causal, n U[1024, 8192]",
+            "kernel": "mla_decode_ragged (attention + combine)", "bound": bound, "achieved": achieved,
+            "peak": tc if bound == "tensor" else hbm, "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
+            "frac": roof / (ms * 1e-3), "peak_source": f"{src}", "call_avg_us": ms * 1e3,
+            "roofline_us": roof * 1e6, "steps": steps}
+
+
 def prefill_work(S, H):
     """Operations of the causal quantised prefill: 2 (192 + 128) per (head, query,
     visible key), S (S + 1) / 2 visible pairs per head."""
@@ -508,6 +583,8 @@ def main():
     ap.add_argument("--prefill-steps", type=int, default=5,
                     help="timed runs of the quantised 64K-token prefill (0 = skip)")
     ap.add_argument("--prefill-shape", default="65536,16", help="S,H of the quantised prefill")
+    ap.add_argument("--ragged-steps", type=int, default=30,
+                    help="timed calls of the ragged-query-count MTP verification (0 = skip)")
     ap.add_argument("--absorb-steps", type=int, default=30,
                     help="timed calls of each absorption GEMM at the serving shape (0 = skip)")
     ap.add_argument("--kv-format", default="bf16", choices=["bf16", "fp8"],
@@ -645,6 +722,10 @@ def main():
             per_workload[name + "_fp8"] = roofline(wi, ti, args.per_workload_steps, fp8=True)
             del ri
             torch.cuda.empty_cache()
+
+    if world == 1 and args.ragged_steps > 0:
+        per_workload["mtp_b128_sq4_ragged"] = bench_ragged(mla, dev, args.ragged_steps, args.warmup, flusher)
+        torch.cuda.empty_cache()
 
     if world == 1 and args.absorb_steps > 0:
         per_workload.update(bench_absorb(mla, dev, args.absorb_steps, args.warmup, flusher))
