@@ -86,9 +86,11 @@ def ragged_work(seqlens, q_lens, H, causal, row_bytes=D_QK * 2):
 def bench_ragged(mla, dev, steps, warmup, flush, B=128, s_q=4, H=128, seed=1005):
     """Speculative-decoding verification with per-sequence accepted drafts: B = 128
     sequences, up to s_q = 4 query tokens each with q_lens[b] drawn uniformly from
-    1..4, causal, lengths U[1024, 8192] as in the MTP workload.  Times the public
-    mla_decode_ragged call (attention and LSE combine) after an L2 flush; the roofline
-    is the slower of the cache bytes at HBM bandwidth and the FLOPs at the bf16 peak."""
+    1..4, causal, lengths U[1024, 8192] as in the MTP workload.  Times two public
+    calls (attention and LSE combine, after an L2 flush): mla_decode_ragged over the
+    per-sequence schedule and mla_decode_tokens over the token schedule (one s_q = 1
+    sequence per query token).  The roofline is the slower of the cache bytes at HBM
+    bandwidth and the FLOPs at the bf16 peak.  Returns {name: entry}."""
     import torch
     from deepseek_mla_decode_b200.workloads import make_inputs
 
@@ -105,37 +107,49 @@ def bench_ragged(mla, dev, steps, warmup, flush, B=128, s_q=4, H=128, seed=1005)
     lens = torch.from_numpy(inp.cache_seqlens).to(dev)
     qls = torch.from_numpy(q_lens).to(dev)
     st = torch.cuda.current_stream()
-    meta = mla.get_metadata(lens, s_q, H, stream=st)
-    ws = torch.empty(mla.workspace_size(B, s_q, H), dtype=torch.uint8, device=dev)
     out = torch.empty((B, s_q, H, 512), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((B, s_q, H), dtype=torch.float32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    for _ in range(warmup):
-        mla.decode_ragged(q_nope, q_pe, kv, table, lens, qls, inp.softmax_scale, True, meta, workspace=ws, out=out,
-                          lse=lse, status=status, stream=st)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
-    for e in ev:
-        flush()
-        e[0].record(st)
-        mla.decode_ragged(q_nope, q_pe, kv, table, lens, qls, inp.softmax_scale, True, meta, workspace=ws, out=out,
-                          lse=lse, status=status, stream=st)
-        e[1].record(st)
-    torch.cuda.synchronize()
-    if int(status.item()) != 0:
-        raise RuntimeError(f"device status {int(status.item())} in the ragged decode")
-    ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
     hbm, tc, _, src = load_peaks()
     flops, cache_bytes, _ = ragged_work(seqlens, q_lens, H, True)
     t_hbm, t_tc = cache_bytes / (hbm * 1e9), flops / (tc * 1e12)
     bound = "tensor" if t_tc >= t_hbm else "hbm"
     roof = max(t_hbm, t_tc)
-    achieved = flops / (ms * 1e-3) / 1e12 if bound == "tensor" else cache_bytes / (ms * 1e-3) / 1e9
-    return {"workload": f"ragged MTP verification B={B}, s_q<={s_q} (q_lens U[1, {s_q}], mean "
-                        f"{float(q_lens.mean()):.2f}), H={H}, causal, n U[1024, 8192]",
-            "kernel": "mla_decode_ragged (attention + combine)", "bound": bound, "achieved": achieved,
-            "peak": tc if bound == "tensor" else hbm, "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
-            "frac": roof / (ms * 1e-3), "peak_source": f"{src}", "call_avg_us": ms * 1e3,
-            "roofline_us": roof * 1e6, "steps": steps}
+    res = {}
+    for name, call in (("mtp_b128_sq4_ragged", "mla_decode_tokens (token schedule; attention + combine)"),
+                       ("mtp_b128_sq4_ragged_tiles", "mla_decode_ragged (per-sequence schedule; attention + combine)")):
+        tokens = name == "mtp_b128_sq4_ragged"
+        if tokens:
+            meta = mla.get_metadata_tokens(lens, qls, s_q, H, True, stream=st)
+            ws = torch.empty(mla.workspace_size(B * s_q, 1, H), dtype=torch.uint8, device=dev)
+            fn = mla.decode_tokens
+        else:
+            meta = mla.get_metadata(lens, s_q, H, stream=st)
+            ws = torch.empty(mla.workspace_size(B, s_q, H), dtype=torch.uint8, device=dev)
+            fn = mla.decode_ragged
+        for _ in range(warmup):
+            fn(q_nope, q_pe, kv, table, lens, qls, inp.softmax_scale, True, meta, workspace=ws, out=out, lse=lse,
+               status=status, stream=st)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for e in ev:
+            flush()
+            e[0].record(st)
+            fn(q_nope, q_pe, kv, table, lens, qls, inp.softmax_scale, True, meta, workspace=ws, out=out, lse=lse,
+               status=status, stream=st)
+            e[1].record(st)
+        torch.cuda.synchronize()
+        if int(status.item()) != 0:
+            raise RuntimeError(f"device status {int(status.item())} in the ragged decode ({name})")
+        ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+        achieved = flops / (ms * 1e-3) / 1e12 if bound == "tensor" else cache_bytes / (ms * 1e-3) / 1e9
+        res[name] = {"workload": f"ragged MTP verification B={B}, s_q<={s_q} (q_lens U[1, {s_q}], mean "
+                                 f"{float(q_lens.mean()):.2f}), H={H}, causal, n U[1024, 8192]",
+                     "kernel": call, "bound": bound, "achieved": achieved,
+                     "peak": tc if bound == "tensor" else hbm, "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
+                     "frac": roof / (ms * 1e-3), "peak_source": f"{src}", "call_avg_us": ms * 1e3,
+                     "roofline_us": roof * 1e6, "steps": steps}
+        del ws
+    return res
 
 
 def prefill_work(S, H):
@@ -724,7 +738,7 @@ def main():
             torch.cuda.empty_cache()
 
     if world == 1 and args.ragged_steps > 0:
-        per_workload["mtp_b128_sq4_ragged"] = bench_ragged(mla, dev, args.ragged_steps, args.warmup, flusher)
+        per_workload.update(bench_ragged(mla, dev, args.ragged_steps, args.warmup, flusher))
         torch.cuda.empty_cache()
 
     if world == 1 and args.absorb_steps > 0:

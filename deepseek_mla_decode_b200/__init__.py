@@ -46,6 +46,9 @@ EXPORTED_SYMBOLS = (
     "mla_sage_quantize",
     "mla_sage_attention",
     "mla_sage_prefill",
+    "mla_get_metadata_tokens",
+    "mla_decode_tokens",
+    "mla_decode_fp8_tokens",
 )
 
 _lib = None
@@ -91,7 +94,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for fn in (L.mla_decode, L.mla_decode_attention):
         fn.restype = c_int
         fn.argtypes = dec_args
-    for fn in (L.mla_decode_ragged, L.mla_decode_fp8, L.mla_decode_fp8_attention):
+    L.mla_get_metadata_tokens.restype = c_int
+    L.mla_get_metadata_tokens.argtypes = [c_vp, c_vp, c_int, c_int, c_int, c_int, c_vp, c_size, c_vp]
+    for fn in (L.mla_decode_ragged, L.mla_decode_fp8, L.mla_decode_fp8_attention, L.mla_decode_tokens,
+               L.mla_decode_fp8_tokens):
         fn.restype = c_int
         fn.argtypes = dec_args[:7] + [c_vp] + dec_args[7:]
     for fn in (L.mla_absorb_q, L.mla_absorb_out):
@@ -241,6 +247,57 @@ def decode_fp8(q_nope, q_pe, kv_fp8, block_table, cache_seqlens, softmax_scale: 
     _check("mla_decode_fp8", load_library().mla_decode_fp8(*args[:7], q_lens.data_ptr() if q_lens is not None
                                                            else None, *args[7:]))
     return out, lse
+
+
+def get_metadata_tokens(cache_seqlens, q_lens, s_q: int, H: int, causal: bool, metadata=None, stream=None):
+    """mla_get_metadata_tokens: the token schedule (an s_q = 1 schedule over B * s_q
+    token sequences) for decode_tokens / decode_fp8_tokens; q_lens may be None."""
+    import torch
+
+    B = cache_seqlens.shape[0]
+    nbytes = metadata_size(B * s_q, 1, H)
+    if metadata is None:
+        metadata = torch.empty((nbytes + 3) // 4, dtype=torch.int32, device=cache_seqlens.device)
+    if q_lens is not None and not q_lens.is_contiguous():
+        raise ValueError("q_lens must be contiguous")
+    _check("mla_get_metadata_tokens", load_library().mla_get_metadata_tokens(
+        cache_seqlens.data_ptr(), q_lens.data_ptr() if q_lens is not None else None, B, s_q, H, int(bool(causal)),
+        metadata.data_ptr(), metadata.numel() * metadata.element_size(), _stream_ptr(stream)))
+    return metadata
+
+
+def _decode_tokens(fn, q_nope, q_pe, kv, block_table, cache_seqlens, q_lens, softmax_scale, causal, metadata,
+                   workspace, out, lse, status, stream):
+    import torch
+
+    B, s_q, H, _ = q_nope.shape
+    if workspace is None:
+        workspace = torch.empty(workspace_size(B * s_q, 1, H), dtype=torch.uint8, device=q_nope.device)
+    _, out, lse = _alloc_outputs(q_nope, workspace, out, lse)
+    if q_lens is not None and not q_lens.is_contiguous():
+        raise ValueError("q_lens must be contiguous")
+    args = _decode_args(q_nope, q_pe, kv, block_table, cache_seqlens, softmax_scale, causal, metadata, workspace,
+                        out, lse, status, stream)
+    qptr = q_lens.data_ptr() if q_lens is not None else None
+    _check(fn, getattr(load_library(), fn)(*args[:7], qptr, *args[7:]))
+    return out, lse
+
+
+def decode_tokens(q_nope, q_pe, kv_cache, block_table, cache_seqlens, q_lens, softmax_scale: float, causal: bool,
+                  metadata, workspace=None, out=None, lse=None, status=None, stream=None) -> Tuple[object, object]:
+    """mla_decode_tokens: decode_ragged balanced by the token schedule (metadata from
+    get_metadata_tokens with the same q_lens and causal flag)."""
+    return _decode_tokens("mla_decode_tokens", q_nope, q_pe, kv_cache, block_table, cache_seqlens, q_lens,
+                          softmax_scale, causal, metadata, workspace, out, lse, status, stream)
+
+
+def decode_fp8_tokens(q_nope, q_pe, kv_fp8, block_table, cache_seqlens, q_lens, softmax_scale: float, causal: bool,
+                      metadata, workspace=None, out=None, lse=None, status=None, stream=None) -> Tuple[object, object]:
+    """mla_decode_fp8_tokens: decode_fp8 with the token schedule."""
+    if kv_fp8.shape[-1] != 656:
+        raise ValueError("packed FP8 cache [num_blocks, 64, 656] expected")
+    return _decode_tokens("mla_decode_fp8_tokens", q_nope, q_pe, kv_fp8, block_table, cache_seqlens, q_lens,
+                          softmax_scale, causal, metadata, workspace, out, lse, status, stream)
 
 
 def decode_fp8_attention(q_nope, q_pe, kv_fp8, block_table, cache_seqlens, softmax_scale: float, causal: bool,

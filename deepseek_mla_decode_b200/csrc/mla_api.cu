@@ -12,11 +12,13 @@
 #include "../../include/mla_decode.h"
 
 namespace mla {
+// tok_* / q_lens + rep: the token schedule (s_q = 1 over B * rep token sequences; see
+// token_seq_len in mla_internal.h); zero / null for the per-sequence schedule.
 cudaError_t launch_metadata(const int32_t* seqlens, int B, int s_q, int H, int num_workers, int32_t* meta,
-                            cudaStream_t stream);
+                            cudaStream_t stream, const int32_t* q_lens = nullptr, int rep = 0, int causal = 0);
 cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, const int32_t* q_lens, int max_blocks,
                            int B, int s_q, int M, int P, const float* part_o, const float* part_lse, void* out,
-                           float* lse, cudaStream_t stream);
+                           float* lse, cudaStream_t stream, int tok_rep = 0, int tok_causal = 0);
 cudaError_t decode_kernel_setup(int device);
 namespace sage {
 cudaError_t attention_setup();
@@ -32,7 +34,8 @@ cudaError_t launch_decode(bool fp8, const CUtensorMap& tm_kv, const CUtensorMap&
                           const int32_t* q_lens, const int32_t* meta, int64_t num_blocks, int B, int s_q,
                           int H, float scale, int causal, void* out, float* lse, float* part_o, float* part_lse,
                           int32_t* status, int num_ctas, uint64_t wait_timeout_ns, int inject_stall,
-                          cudaStream_t stream);
+                          cudaStream_t stream, int tok_rep = 0, int tok_causal = 0,
+                          const int32_t* tok_q_lens = nullptr);
 }  // namespace mla
 
 namespace {
@@ -269,7 +272,8 @@ mla_status_t launch_attention(bool fp8, const void* q_nope, const void* q_pe, co
                               int64_t num_blocks, const int32_t* block_table, int max_blocks,
                               const int32_t* cache_seqlens, const int32_t* q_lens, int B, int s_q, int H,
                               float softmax_scale, int causal, const void* metadata, void* workspace, void* out,
-                              float* lse, int32_t* status, const DecodeGeom& g, cudaStream_t s) {
+                              float* lse, int32_t* status, const DecodeGeom& g, cudaStream_t s, int tok_rep = 0,
+                              int tok_causal = 0, const int32_t* tok_q_lens = nullptr) {
   const int64_t rows = static_cast<int64_t>(B) * g.M;
   CUtensorMap tm_kv, tm_kv2, tm_qn, tm_qp, tm_kpe, tm_scl;
   if (fp8) {
@@ -324,7 +328,8 @@ mla_status_t launch_attention(bool fp8, const void* q_nope, const void* q_pe, co
                          tm_out, tm_part, block_table, max_blocks, cache_seqlens,
                          q_lens, static_cast<const int32_t*>(metadata), num_blocks, B, s_q, H, softmax_scale,
                          causal != 0,
-                         out, lse, part_o, part_lse, status, 2 * g.P * g.T, g_wait_timeout_ns.load(), g_inject_stall.load(), s) != cudaSuccess)
+                         out, lse, part_o, part_lse, status, 2 * g.P * g.T, g_wait_timeout_ns.load(), g_inject_stall.load(), s,
+                         tok_rep, tok_causal, tok_q_lens) != cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;
 }
@@ -393,25 +398,35 @@ mla_status_t mla_decode(const void* q_nope, const void* q_pe, const void* kv_cac
 namespace {
 
 // Validation, attention and combine launches shared by the bf16 and FP8 entry points.
+// tokens: the token schedule, an s_q = 1 decode over B * s_q token sequences (q, out
+// and lse are the same memory viewed as [B * s_q, 1, H, ...]); the metadata must come
+// from mla_get_metadata_tokens with the same q_lens and causal flag.
 mla_status_t decode_any(bool fp8, const void* q_nope, const void* q_pe, const void* kv_cache, int64_t num_blocks,
                         const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
                         const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
                         const void* metadata, size_t metadata_bytes, void* workspace, size_t workspace_bytes,
-                        void* out, float* lse, int32_t* status, void* stream) {
+                        void* out, float* lse, int32_t* status, void* stream, bool tokens = false) {
   if (q_lens && (reinterpret_cast<uintptr_t>(q_lens) & 3u)) return MLA_ERR_INVALID_ARG;
+  if (tokens && !shape_supported(B, s_q, H)) return MLA_ERR_UNSUPPORTED;
+  const int Bl = tokens ? B * s_q : B, sl = tokens ? 1 : s_q;  // the launch's batch and query count
   DecodeGeom g;
   mla_status_t st = check_decode_args(q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens,
-                                      B, s_q, H, softmax_scale, metadata, metadata_bytes, workspace,
+                                      Bl, sl, H, softmax_scale, metadata, metadata_bytes, workspace,
                                       workspace_bytes, out, lse, status, &g);
   if (st != MLA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_attention(fp8, q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, q_lens, B,
-                        s_q, H, softmax_scale, causal, metadata, workspace, out, lse, status, g, s);
+  if (tokens)
+    st = launch_attention(fp8, q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, nullptr,
+                          Bl, 1, H, softmax_scale, 0, metadata, workspace, out, lse, status, g, s, s_q,
+                          causal != 0, q_lens);
+  else
+    st = launch_attention(fp8, q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, q_lens,
+                          B, s_q, H, softmax_scale, causal, metadata, workspace, out, lse, status, g, s);
   if (st != MLA_OK) return st;
   const float* part_o = static_cast<const float*>(workspace);
   const float* part_lse = part_o + g.slots * g.M * mla::kDLatent;
-  if (mla::launch_combine(static_cast<const int32_t*>(metadata), cache_seqlens, q_lens, max_blocks, B, s_q, g.M,
-                          g.P, part_o, part_lse, out, lse, s) != cudaSuccess)
+  if (mla::launch_combine(static_cast<const int32_t*>(metadata), cache_seqlens, q_lens, max_blocks, Bl, sl, g.M,
+                          g.P, part_o, part_lse, out, lse, s, tokens ? s_q : 0, tokens && causal != 0) != cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;
 }
@@ -438,6 +453,45 @@ mla_status_t mla_decode_fp8(const void* q_nope, const void* q_pe, const void* kv
   return decode_any(true, q_nope, q_pe, kv_fp8, num_blocks, block_table, max_blocks, cache_seqlens, q_lens, B,
                     s_q, H, softmax_scale, causal, metadata, metadata_bytes, workspace, workspace_bytes, out, lse,
                     status, stream);
+}
+
+mla_status_t mla_get_metadata_tokens(const int32_t* cache_seqlens, const int32_t* q_lens, int B, int s_q, int H,
+                                     int causal, void* metadata, size_t metadata_bytes, void* stream) {
+  if (!cache_seqlens || !metadata) return MLA_ERR_INVALID_ARG;
+  if (!shape_supported(B, s_q, H) || !shape_supported(B * s_q, 1, H)) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(metadata) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(q_lens) & 3u))
+    return MLA_ERR_INVALID_ARG;
+  size_t need = 0;
+  mla_metadata_size(B * s_q, 1, H, &need);
+  if (metadata_bytes < need) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  mla_status_t st = device_info(&sms);
+  if (st != MLA_OK) return st;
+  if (mla::launch_metadata(cache_seqlens, B * s_q, 1, H, num_workers_for(sms), static_cast<int32_t*>(metadata),
+                           static_cast<cudaStream_t>(stream), q_lens, s_q, causal != 0) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+mla_status_t mla_decode_tokens(const void* q_nope, const void* q_pe, const void* kv_cache, int64_t num_blocks,
+                               const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                               const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
+                               const void* metadata, size_t metadata_bytes, void* workspace,
+                               size_t workspace_bytes, void* out, float* lse, int32_t* status, void* stream) {
+  return decode_any(false, q_nope, q_pe, kv_cache, num_blocks, block_table, max_blocks, cache_seqlens, q_lens, B,
+                    s_q, H, softmax_scale, causal, metadata, metadata_bytes, workspace, workspace_bytes, out, lse,
+                    status, stream, true);
+}
+
+mla_status_t mla_decode_fp8_tokens(const void* q_nope, const void* q_pe, const void* kv_fp8, int64_t num_blocks,
+                                   const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                                   const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
+                                   const void* metadata, size_t metadata_bytes, void* workspace,
+                                   size_t workspace_bytes, void* out, float* lse, int32_t* status, void* stream) {
+  return decode_any(true, q_nope, q_pe, kv_fp8, num_blocks, block_table, max_blocks, cache_seqlens, q_lens, B,
+                    s_q, H, softmax_scale, causal, metadata, metadata_bytes, workspace, workspace_bytes, out, lse,
+                    status, stream, true);
 }
 
 mla_status_t mla_decode_fp8_attention(const void* q_nope, const void* q_pe, const void* kv_fp8, int64_t num_blocks,

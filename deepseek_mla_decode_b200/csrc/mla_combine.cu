@@ -39,7 +39,7 @@ template <int kColParts, int kGroup>
 __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
     const int32_t* __restrict__ meta, const int32_t* __restrict__ seqlens, const int32_t* __restrict__ q_lens,
     int max_blocks, int B, int s_q, int M, const float* __restrict__ part_o, const float* __restrict__ part_lse,
-    __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+    __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int tok_rep, int tok_causal) {
   // launched as a programmatic dependent of the attention kernel: wait for it
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int part = blockIdx.x;
@@ -54,8 +54,16 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
   const int nblk = meta[off_nblk() + b];
   const int ns = meta[off_num_splits(B) + b];
   const int slot0 = meta[off_split_prefix(B) + b];
-  const int n = seqlens[b];
-  const int ql = (q_lens != nullptr) ? q_lens[b] : s_q;
+  // with a token schedule, sequence b is one token of real sequence b / tok_rep (its
+  // length from token_seq_len, one query token)
+  const int r = tok_rep ? b / tok_rep : b;
+  const int nr = seqlens[r];
+  const int qr = (q_lens != nullptr) ? q_lens[r] : (tok_rep ? tok_rep : s_q);
+  const int n = !tok_rep ? nr
+                         : ((int64_t)nr > (int64_t)max_blocks * kBlockSize ? -1
+                                                                            : token_seq_len(nr, qr, b - r * tok_rep, tok_rep,
+                                                                                            tok_causal));
+  const int ql = tok_rep ? 1 : qr;
   if (fp + 1 != part) return;  // a later cut of the same sequence
   // rows written as NaN already: invalid length, or a schedule built for another length
   if (n < 0 || (int64_t)n > (int64_t)max_blocks * kBlockSize) return;
@@ -142,7 +150,7 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
 
 cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, const int32_t* q_lens, int max_blocks,
                            int B, int s_q, int M, int P, const float* part_o, const float* part_lse, void* out, float* lse,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, int tok_rep, int tok_causal) {
   // few sequences: long ones with many splits and few rows to merge
   const bool wide = B < kWideBatch;
   const int parts = wide ? 4 : 1;
@@ -158,9 +166,9 @@ cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, const in
   cfg.numAttrs = 1;
   if (wide)
     return cudaLaunchKernelEx(&cfg, combine_kernel<4, 8>, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o,
-                              part_lse, reinterpret_cast<__nv_bfloat16*>(out), lse);
+                              part_lse, reinterpret_cast<__nv_bfloat16*>(out), lse, tok_rep, tok_causal);
   return cudaLaunchKernelEx(&cfg, combine_kernel<1, 2>, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o, part_lse,
-                            reinterpret_cast<__nv_bfloat16*>(out), lse);
+                            reinterpret_cast<__nv_bfloat16*>(out), lse, tok_rep, tok_causal);
 }
 
 }  // namespace mla

@@ -116,6 +116,11 @@ struct Params {
   const int32_t* block_table;
   const int32_t* seqlens;
   const int32_t* q_lens;  // per-sequence query tokens (<= s_q), or null: s_q for every sequence
+  // Token schedule (tok_rep > 0): the launch is an s_q = 1 decode of B = B_real * tok_rep
+  // sequences; sequence u is token u % tok_rep of real sequence u / tok_rep, whose
+  // length, table row and query count (tok_q_lens, or tok_rep each) it takes.
+  const int32_t* tok_q_lens;
+  int tok_rep, tok_causal;
   const int32_t* meta;
   __nv_bfloat16* out;
   float* lse;
@@ -162,6 +167,21 @@ struct Piece {
   int b, k_lo, k_hi, split, n, qlen;
 };
 
+// Keys of sequence u: its length, or with a token schedule the length of token
+// u % tok_rep of its real sequence (token_seq_len; a real length beyond the table makes
+// every token of that sequence invalid, as the real sequence would be).
+__device__ __forceinline__ int seq_len(const Params& p, int u) {
+  if (p.tok_rep == 0) return p.seqlens[u];
+  const int r = u / p.tok_rep;
+  const int n = p.seqlens[r];
+  if ((int64_t)n > (int64_t)p.max_blocks * kBlockSize) return -1;
+  return token_seq_len(n, p.tok_q_lens ? p.tok_q_lens[r] : p.tok_rep, u - r * p.tok_rep, p.tok_rep, p.tok_causal);
+}
+// Block-table row of sequence u.
+__device__ __forceinline__ int64_t table_row(const Params& p, int u) {
+  return p.tok_rep ? u / p.tok_rep : u;
+}
+
 // Block count of a sequence of n keys, or -1 when n is not a valid length for the table.
 __device__ __forceinline__ int expected_blocks(const Params& p, int n) {
   if (n < 0 || (int64_t)n > (int64_t)p.max_blocks * kBlockSize) return -1;
@@ -207,7 +227,7 @@ struct PieceWalker {
       cb += 1;
       ck = 0;
       if (lo >= hi) continue;
-      const int n = p->seqlens[b];
+      const int n = seq_len(*p, b);
       if (expected_blocks(*p, n) != nb) continue;
       const int ql = query_len(*p, b);
       if (ql < 0 || row0 >= ql * p->H) continue;
@@ -415,7 +435,7 @@ __device__ __forceinline__ int clamp_block_id(const Params& p, int32_t id) {
 __device__ __forceinline__ void write_orphan_rows(const Params& p, int part, int P, int row0, int y0, int lane) {
   const int32_t* nblk = p.meta + off_nblk();
   for (int b = part; b < p.B; b += P) {
-    const int n = p.seqlens[b];
+    const int n = seq_len(p, b);
     const int want = expected_blocks(p, n);
     const int ql = query_len(p, b);
     const bool bad_len = want < 0 || ql < 0;
@@ -517,7 +537,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
   const int P = p.meta[kHdrNumParts];
   int T = p.meta[kHdrNumTiles];
   if (p.meta[kHdrMagic] != kMetaMagic || p.meta[kHdrB] != p.B || p.meta[kHdrSq] != p.s_q ||
-      p.meta[kHdrH] != p.H || P * T * 2 != (int)gridDim.x) {
+      p.meta[kHdrH] != p.H || P * T * 2 != (int)gridDim.x || p.meta[kHdrTokens] != p.tok_rep ||
+      (p.tok_rep != 0 && p.meta[kHdrTokCausal] != p.tok_causal)) {
     if (tid == 0 && blockIdx.x == 0) set_status(p, kErrMetadata);
     T = 0;  // every role skips; the CTA still joins the cluster barriers below
   }
@@ -705,7 +726,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
       bool have = walk.next(cur);
       bool have_nxt = have && walk.next(nxt);
       if (have) {
-        bt = p.block_table + (int64_t)cur.b * p.max_blocks;
+        bt = p.block_table + table_row(p, cur.b) * p.max_blocks;
         id_pending = fetch_id(lane);
       }
       while (ok && have) {
@@ -714,7 +735,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
         int id_next = 0;
         for (int t = 0; t < nt && ok; ++t) {
           if (t == nt - 1 && have_nxt) {
-            const int32_t* btn = p.block_table + (int64_t)nxt.b * p.max_blocks;
+            const int32_t* btn = p.block_table + table_row(p, nxt.b) * p.max_blocks;
             id_next = (lane < nxt.k_hi - nxt.k_lo) ? clamp_block_id(p, btn[nxt.k_lo + lane]) : 0;
           }
           if (t == 0 && pi == 0) load_q(cur, npieces);
@@ -734,7 +755,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
         have = have_nxt;
         if (have) {
           cur = nxt;
-          bt = p.block_table + (int64_t)cur.b * p.max_blocks;
+          bt = p.block_table + table_row(p, cur.b) * p.max_blocks;
           id_pending = id_next;
           have_nxt = walk.next(nxt);
         }
@@ -971,7 +992,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<kFp8>::kThreads,
         const int split_base = p.meta[off_split_prefix(p.B) + pc.b];
         int bad_ids = 0;
         {
-          const int32_t* bt = p.block_table + (int64_t)pc.b * p.max_blocks;
+          const int32_t* bt = p.block_table + table_row(p, pc.b) * p.max_blocks;
           for (int k = pc.k_lo + st; k < pc.k_hi; k += kNumSoftmaxThreads) {
             const int32_t id = bt[k];
             bad_ids |= (id < 0 || (int64_t)id >= p.num_blocks);
@@ -1436,7 +1457,7 @@ cudaError_t launch_decode(bool fp8, const CUtensorMap& tm_kv, const CUtensorMap&
                           const int32_t* q_lens, const int32_t* meta, int64_t num_blocks, int B, int s_q,
                           int H, float scale, int causal, void* out, float* lse, float* part_o, float* part_lse,
                           int32_t* status, int num_ctas, uint64_t wait_timeout_ns, int inject_stall,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, int tok_rep, int tok_causal, const int32_t* tok_q_lens) {
   if (fp8 && (!tm_kpe || !tm_scl)) return cudaErrorInvalidValue;
   Params prm;
   std::memset(&prm, 0, sizeof(prm));
@@ -1453,6 +1474,9 @@ cudaError_t launch_decode(bool fp8, const CUtensorMap& tm_kv, const CUtensorMap&
   prm.block_table = block_table;
   prm.seqlens = seqlens;
   prm.q_lens = q_lens;
+  prm.tok_q_lens = tok_q_lens;
+  prm.tok_rep = tok_rep;
+  prm.tok_causal = tok_causal;
   prm.meta = meta;
   prm.out = reinterpret_cast<__nv_bfloat16*>(out);
   prm.lse = lse;

@@ -43,8 +43,24 @@ enum HdrField : int {
   kHdrTotalSlots = 7, // sum of num_splits
   kHdrNumWorkers = 8, // CTA pairs available on the device
   kHdrOverhead = 9,
+  kHdrTokens = 10,    // token schedule: the call's s_q (query tokens per sequence); 0 otherwise
+  kHdrTokCausal = 11, // token schedule: the causal flag the lengths were built with
 };
 constexpr int32_t kMetaMagic = 0x4D4C4131;  // "MLA1"
+
+// Token schedule: the decode of B sequences with up to `rep` query tokens each (q of
+// them real) runs as an s_q = 1 decode of B * rep sequences; sequence u = b * rep + t
+// is token t of b.  With the causal mask token t sees the first n - q + t + 1 keys of
+// b (all n without it); a padding token (t >= q) sees none.  -1 marks an invalid query
+// count or a negative length.  The schedule, the attention kernel and the combine all
+// take a token's length from here.
+__host__ __device__ inline int token_seq_len(int n, int q, int t, int rep, int causal) {
+  if (q < 0 || q > rep || n < 0) return -1;
+  if (t >= q) return 0;
+  if (!causal) return n;
+  const int v = n - q + t + 1;
+  return v > 0 ? v : 0;
+}
 
 __host__ __device__ inline int64_t meta_words(int B) {
   return kHdrWords + 4LL * kMaxWorkers + 4LL * B;

@@ -49,8 +49,21 @@ __device__ int64_t block_exclusive_scan(int64_t v, int64_t* scratch /*[32]*/, in
 
 // kThreads = 256 for batches of at most 256 sequences (fewer and cheaper block-wide
 // barriers), 1024 otherwise.
+// Length of sequence b: seqlens[b], or with a token schedule (rep > 0) the length of
+// virtual sequence b = token b % rep of real sequence b / rep (token_seq_len).
+struct Lengths {
+  const int32_t* seqlens;
+  const int32_t* q_lens;  // token schedule: per-sequence query counts, or null (rep each)
+  int rep, causal;
+  __device__ int operator()(int b) const {
+    if (rep == 0) return seqlens[b];
+    const int r = b / rep;
+    return token_seq_len(seqlens[r], q_lens ? q_lens[r] : rep, b - r * rep, rep, causal);
+  }
+};
+
 template <int kThreads>
-__global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __restrict__ seqlens, int B,
+__global__ void __launch_bounds__(kThreads) metadata_kernel(const Lengths len_of, int B,
                                                             int s_q, int H, int num_workers,
                                                             int32_t* __restrict__ meta) {
   __shared__ int64_t scratch[32];
@@ -76,7 +89,7 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
   // one scan of the costs instead of two)
   if (B <= kThreads) {
     const int b = tid;
-    const int n = (b < B) ? seqlens[b] : 0;
+    const int n = (b < B) ? len_of(b) : 0;
     const int nb = n > 0 ? (n + kBlockSize - 1) / kBlockSize : 0;
     const int64_t nt = (nb + kBlocksPerTile - 1) / kBlocksPerTile;
     const int64_t cost = nb > 0 ? nt + kSchedOverheadTiles : 0;
@@ -135,6 +148,8 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
       meta[kHdrNumWorkers] = num_workers;
       meta[kHdrOverhead] = kSchedOverheadTiles;
       for (int i = kHdrOverhead + 1; i < kHdrWords; ++i) meta[i] = 0;
+      meta[kHdrTokens] = len_of.rep;
+      meta[kHdrTokCausal] = len_of.rep ? len_of.causal : 0;
     }
     return;
   }
@@ -145,7 +160,7 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
     const int b = base + tid;
     int64_t cost = 0;
     if (b < B) {
-      const int n = seqlens[b];
+      const int n = len_of(b);
       const int nb = n > 0 ? (n + kBlockSize - 1) / kBlockSize : 0;
       nblk_out[b] = nb;
       cost = nb > 0 ? (nb + kBlocksPerTile - 1) / kBlocksPerTile + kSchedOverheadTiles : 0;
@@ -171,7 +186,7 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
     int64_t cost = 0;
     int nb = 0;
     if (b < B) {
-      const int n = seqlens[b];
+      const int n = len_of(b);
       nb = n > 0 ? (n + kBlockSize - 1) / kBlockSize : 0;
       cost = nb > 0 ? (nb + kBlocksPerTile - 1) / kBlocksPerTile + kSchedOverheadTiles : 0;
     }
@@ -241,17 +256,20 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
     meta[kHdrNumWorkers] = num_workers;
     meta[kHdrOverhead] = kSchedOverheadTiles;
     for (int i = kHdrOverhead + 1; i < kHdrWords; ++i) meta[i] = 0;
+    meta[kHdrTokens] = len_of.rep;
+    meta[kHdrTokCausal] = len_of.rep ? len_of.causal : 0;
   }
 }
 
 }  // namespace
 
 cudaError_t launch_metadata(const int32_t* seqlens, int B, int s_q, int H, int num_workers,
-                            int32_t* meta, cudaStream_t stream) {
+                            int32_t* meta, cudaStream_t stream, const int32_t* q_lens, int rep, int causal) {
+  const Lengths len_of{seqlens, q_lens, rep, causal};
   if (B <= 256)
-    metadata_kernel<256><<<1, 256, 0, stream>>>(seqlens, B, s_q, H, num_workers, meta);
+    metadata_kernel<256><<<1, 256, 0, stream>>>(len_of, B, s_q, H, num_workers, meta);
   else
-    metadata_kernel<1024><<<1, 1024, 0, stream>>>(seqlens, B, s_q, H, num_workers, meta);
+    metadata_kernel<1024><<<1, 1024, 0, stream>>>(len_of, B, s_q, H, num_workers, meta);
   return cudaGetLastError();
 }
 

@@ -162,6 +162,43 @@ mla_status_t mla_decode_ragged(const void* q_nope, const void* q_pe, const void*
                                void* out, float* lse, int32_t* status, void* stream);
 
 /*
+ * Token schedule for ragged query counts.  mla_decode_ragged schedules every 128-row
+ * tile of query rows over the same partitions, so when sequences carry different
+ * numbers of real tokens the tiles of the later token positions (held only by the
+ * sequences that kept that many drafts) leave their partitions' CTAs idle.  The token
+ * schedule instead runs the call as an s_q = 1 decode over B * s_q token sequences:
+ * sequence u = b * s_q + t is token t of sequence b, with the first n_b - q_lens[b] + t + 1
+ * keys of b under the causal mask (all n_b keys without it) and none for a padding
+ * token (t >= q_lens[b]).  That is the same result (the causal mask of a token is a
+ * shorter visible prefix; speculative-decoding section of the Paddle 3.0 inference
+ * upgrade article for the per-sequence draft counts), balanced over all CTAs like an
+ * s_q = 1 batch.
+ *
+ * mla_get_metadata_tokens: the schedule for mla_decode_tokens / mla_decode_fp8_tokens.
+ *   q_lens may be NULL (s_q tokens for every sequence); causal must be the flag the
+ *   decode will use.  metadata holds mla_metadata_size(B * s_q, 1, H) bytes.
+ * mla_decode_tokens, mla_decode_fp8_tokens: arguments and outputs as mla_decode_ragged /
+ *   mla_decode_fp8 (q, out, lse in the padded [B, s_q, H, ...] layout); the metadata must
+ *   come from mla_get_metadata_tokens with the same cache_seqlens, q_lens and causal flag,
+ *   and the workspace holds mla_workspace_size(B * s_q, 1, H) bytes.  Device errors as in
+ *   mla_decode_ragged (an invalid length or query count makes all of that sequence's rows
+ *   NaN and sets MLA_DEVICE_ERR_SEQLEN; metadata of another shape, schedule kind or causal
+ *   flag sets MLA_DEVICE_ERR_METADATA).  Library scheduling, no further passage.
+ */
+mla_status_t mla_get_metadata_tokens(const int32_t* cache_seqlens, const int32_t* q_lens, int B, int s_q, int H,
+                                     int causal, void* metadata, size_t metadata_bytes, void* stream);
+mla_status_t mla_decode_tokens(const void* q_nope, const void* q_pe, const void* kv_cache, int64_t num_blocks,
+                               const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                               const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
+                               const void* metadata, size_t metadata_bytes, void* workspace,
+                               size_t workspace_bytes, void* out, float* lse, int32_t* status, void* stream);
+mla_status_t mla_decode_fp8_tokens(const void* q_nope, const void* q_pe, const void* kv_fp8, int64_t num_blocks,
+                                   const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                                   const int32_t* q_lens, int B, int s_q, int H, float softmax_scale, int causal,
+                                   const void* metadata, size_t metadata_bytes, void* workspace,
+                                   size_t workspace_bytes, void* out, float* lse, int32_t* status, void* stream);
+
+/*
  * The two launches mla_decode performs, exposed separately (same arguments, same
  * semantics; mla_decode == mla_decode_attention followed by mla_decode_combine on
  * the same stream with the same workspace).
