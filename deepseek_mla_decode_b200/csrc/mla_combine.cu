@@ -10,9 +10,12 @@
 // flight; batches of few sequences (long ones, cut into many splits, few rows) take
 // four warps per row, each over 128 columns with eight splits in flight.
 //
-// Grid (P, ceil(M * c / 8)), c warps per row: block x = p looks at partition p's first block; a split
-// sequence is exactly one whose cut opens a partition mid-sequence, and the first such
-// partition (first_part + 1) owns its merge, so only blocks with work touch memory.
+// Grid (X, ceil(M * c / 8)), c warps per row.  With more sequences than partitions,
+// X = P and block x = p looks at partition p's first block: a split sequence is
+// exactly one whose cut opens a partition mid-sequence, and the first such partition
+// (first_part + 1) owns its merge, so only blocks with work read more.  With no more
+// sequences than partitions, X = B and block x = b takes sequence b if it has two or
+// more pieces: no idle partitions' blocks, and one round trip less (b is known).
 // Rows of sequences that no partition covers (no visible key, invalid length, a block
 // count in the metadata that does not match the length) are written by the attention
 // kernel.
@@ -34,22 +37,28 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 }
 
 // kColParts warps per query row, each over 512 / kColParts columns; kGroup partial rows
-// in flight per lane (both give 32 registers of loads)
-template <int kColParts, int kGroup>
+// in flight per lane (both give 32 registers of loads); kBySeq: block x is a sequence
+// (else a partition)
+template <int kColParts, int kGroup, bool kBySeq>
 __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
     const int32_t* __restrict__ meta, const int32_t* __restrict__ seqlens, const int32_t* __restrict__ q_lens,
     int max_blocks, int B, int s_q, int M, const float* __restrict__ part_o, const float* __restrict__ part_lse,
     __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int tok_rep, int tok_causal) {
   // launched as a programmatic dependent of the attention kernel: wait for it
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int part = blockIdx.x;
-  if (part == 0) return;
-  // Three dependent round trips to memory: the partition's start, then every word of
-  // its sequence at once, then the partial lse values together with the first
-  // partial rows (the rest of the kernel is arithmetic on registers).
-  const int b = meta[off_part_start() + 2 * part];
-  const int k0 = meta[off_part_start() + 2 * part + 1];
-  if (b >= B || k0 == 0) return;  // partition opens a sequence (or is empty)
+  // Dependent round trips to memory: the partition's start (by partition only), then
+  // every word of the sequence at once, then the partial lse values together with the
+  // first partial rows (the rest of the kernel is arithmetic on registers).
+  int b, part = 0;
+  if constexpr (kBySeq) {
+    b = blockIdx.x;
+  } else {
+    part = blockIdx.x;
+    if (part == 0) return;
+    b = meta[off_part_start() + 2 * part];
+    const int k0 = meta[off_part_start() + 2 * part + 1];
+    if (b >= B || k0 == 0) return;  // partition opens a sequence (or is empty)
+  }
   const int fp = meta[off_first_part(B) + b];
   const int nblk = meta[off_nblk() + b];
   const int ns = meta[off_num_splits(B) + b];
@@ -64,7 +73,11 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
                                                                             : token_seq_len(nr, qr, b - r * tok_rep, tok_rep,
                                                                                             tok_causal));
   const int ql = tok_rep ? 1 : qr;
-  if (fp + 1 != part) return;  // a later cut of the same sequence
+  if constexpr (kBySeq) {
+    if (ns < 2) return;  // one piece: its rows were written by the attention kernel
+  } else {
+    if (fp + 1 != part) return;  // a later cut of the same sequence
+  }
   // rows written as NaN already: invalid length, or a schedule built for another length
   if (n < 0 || (int64_t)n > (int64_t)max_blocks * kBlockSize) return;
   if (nblk != (n + kBlockSize - 1) / kBlockSize) return;
@@ -153,9 +166,10 @@ cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, const in
                            cudaStream_t stream, int tok_rep, int tok_causal) {
   // few sequences: long ones with many splits and few rows to merge
   const bool wide = B < kWideBatch;
+  const bool by_seq = wide || B <= P;
   const int parts = wide ? 4 : 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(P, (M * parts + kWarps - 1) / kWarps);
+  cfg.gridDim = dim3(by_seq ? B : P, (M * parts + kWarps - 1) / kWarps);
   cfg.blockDim = dim3(kWarps * 32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -164,11 +178,15 @@ cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, const in
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
   if (wide)
-    return cudaLaunchKernelEx(&cfg, combine_kernel<4, 8>, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o,
-                              part_lse, reinterpret_cast<__nv_bfloat16*>(out), lse, tok_rep, tok_causal);
-  return cudaLaunchKernelEx(&cfg, combine_kernel<1, 2>, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o, part_lse,
-                            reinterpret_cast<__nv_bfloat16*>(out), lse, tok_rep, tok_causal);
+    return cudaLaunchKernelEx(&cfg, combine_kernel<4, 8, true>, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o,
+                              part_lse, o, lse, tok_rep, tok_causal);
+  if (by_seq)
+    return cudaLaunchKernelEx(&cfg, combine_kernel<1, 2, true>, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o,
+                              part_lse, o, lse, tok_rep, tok_causal);
+  return cudaLaunchKernelEx(&cfg, combine_kernel<1, 2, false>, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o,
+                            part_lse, o, lse, tok_rep, tok_causal);
 }
 
 }  // namespace mla
