@@ -8,7 +8,7 @@
 // partial rows with 16-byte loads and write the bf16 row once.  Batches of many
 // sequences (few splits each, many rows) take one warp per row with two splits in
 // flight; batches of few sequences (long ones, cut into many splits, few rows) take
-// four warps per row, each over 128 columns with eight splits in flight.
+// four warps per row, each over 128 columns with sixteen splits in flight.
 //
 // Grid (X, ceil(M * c / 8)), c warps per row.  With more sequences than partitions,
 // X = P and block x = p looks at partition p's first block: a split sequence is
@@ -37,8 +37,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 }
 
 // kColParts warps per query row, each over 512 / kColParts columns; kGroup partial rows
-// in flight per lane (both give 32 registers of loads); kBySeq: block x is a sequence
-// (else a partition)
+// in flight per lane (32 registers of loads for one warp per row and two splits, 64 for
+// four warps per row and sixteen splits); kBySeq: block x is a sequence (else a
+// partition)
 template <int kColParts, int kGroup, bool kBySeq>
 __global__ void __launch_bounds__(kWarps * 32) combine_kernel(
     const int32_t* __restrict__ meta, const int32_t* __restrict__ seqlens, const int32_t* __restrict__ q_lens,
@@ -180,7 +181,7 @@ cudaError_t launch_combine(const int32_t* meta, const int32_t* seqlens, const in
   cfg.numAttrs = 1;
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
   if (wide)
-    return cudaLaunchKernelEx(&cfg, combine_kernel<4, 8, true>, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o,
+    return cudaLaunchKernelEx(&cfg, combine_kernel<4, 16, true>, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o,
                               part_lse, o, lse, tok_rep, tok_causal);
   if (by_seq)
     return cudaLaunchKernelEx(&cfg, combine_kernel<1, 2, true>, meta, seqlens, q_lens, max_blocks, B, s_q, M, part_o,
