@@ -93,6 +93,19 @@ def test_single_long_sequence_split():
     check(make_inputs(1, 1, 128, [20000], seed=61))
 
 
+@pytest.mark.parametrize("extra", [-1, 0, 1])
+def test_combine_grid_forms_at_the_partition_count(extra):
+    """The combine's grid runs over sequences while B <= P (partitions per row tile) and
+    over partitions beyond: batches of P - 1, P and P + 1 sequences, lengths mixed so
+    that some sequences are cut into two or more pieces and some are whole."""
+    P = min(mla.device_sm_count() // 2, 256)  # CTA pairs = partitions of the single row tile
+    B = P + extra
+    rng = np.random.default_rng(300 + extra)
+    lens = rng.integers(1, 6000, size=B).astype(np.int32)
+    lens[::7] = rng.integers(9000, 20000, size=len(lens[::7]))
+    check(make_inputs(B, 1, 128, lens, seed=301 + extra))
+
+
 def test_nan_poison_outside_visible_range():
     inp = make_inputs(4, 1, 32, [37, 100, 129, 200], seed=62, nan_poison=True)
     check(inp)
